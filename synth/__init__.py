@@ -1,0 +1,99 @@
+"""Seeded synthetic inputs shared by the oracle and the CUDA path.
+
+This package holds shapes and random draws only -- none of the block's
+arithmetic (no quantisation, normalisation, RoPE, attention or GEMM).  Both
+``oracle`` and the tests/bench feed the CUDA library from the same tensors made
+here, so the two sides see identical bytes.
+
+Workloads (token counts from [P4] "Welcome FLUX.3 Image Klein in Diffusers",
+§The VAE and Tokenization -- 8x VAE, 2x2 patches, 1024x1024 -> 64x64 = 4,096
+tokens -- and [P2] "FLUX.3 Image Klein Brings 2-Second AI Image Generation to
+Diffusers", §Summary -- each 1024x1024 reference adds 4,096 tokens; hidden
+width 3072 from [P4] §The Qwen3-VL Text Encoder):
+
+=============  ======  ======  ====  ===  =====  =====  =========
+name           text    grid    refs  D    heads  F      attention
+=============  ======  ======  ====  ===  =====  =====  =========
+micro          16      4x4     1     128  1      384    bf16
+tiny           64      16x16   0     512  4      1536   bf16
+t2i_1024       512     64x64   0     3072 24     9216   fp8
+i2i_1024       512     64x64   1     3072 24     9216   fp8
+multiref_1024  512     64x64   4     3072 24     9216   fp8
+multiref_21504 1024    64x64   4     3072 24     9216   fp8
+=============  ======  ======  ====  ===  =====  =====  =========
+
+Draw recipe (fixed order, one ``torch.Generator`` seeded per workload, every
+tensor ``randn`` in fp32 then cast to bf16 with round-to-nearest-even):
+x ~ N(0, 1) [T, D]; shift1, scale1, gate1, shift2, scale2, gate2 ~ N(0, 0.1)
+[D]; Wqkv [3D, D], Wo [D, D], W1 [2F, D], W2 [D, F] ~ N(0, 0.02).
+"""
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    n_text: int
+    grid_h: int
+    grid_w: int
+    n_ref: int
+    hidden: int
+    heads: int
+    mlp_hidden: int
+    attn: str          # "bf16" or "fp8"
+    seed: int
+
+    @property
+    def n_tokens(self):
+        return self.n_text + (1 + self.n_ref) * self.grid_h * self.grid_w
+
+
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("micro", 16, 4, 4, 1, 128, 1, 384, "bf16", 7),
+        Workload("tiny", 64, 16, 16, 0, 512, 4, 1536, "bf16", 0),
+        Workload("t2i_1024", 512, 64, 64, 0, 3072, 24, 9216, "fp8", 1),
+        Workload("i2i_1024", 512, 64, 64, 1, 3072, 24, 9216, "fp8", 2),
+        Workload("multiref_1024", 512, 64, 64, 4, 3072, 24, 9216, "fp8", 4),
+        Workload("multiref_21504", 1024, 64, 64, 4, 3072, 24, 9216, "fp8", 4),
+    ]
+}
+
+MOD_NAMES = ("shift1", "scale1", "gate1", "shift2", "scale2", "gate2")
+
+
+def _randn(gen, shape, std):
+    return (torch.randn(*shape, generator=gen, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def block_inputs(wl, with_weights=True):
+    """All seeded inputs of one joint-block call, as bf16 CPU tensors."""
+    if isinstance(wl, str):
+        wl = WORKLOADS[wl]
+    g = torch.Generator().manual_seed(wl.seed)
+    T, D, F = wl.n_tokens, wl.hidden, wl.mlp_hidden
+    out = {"x": _randn(g, (T, D), 1.0)}
+    for n in MOD_NAMES:
+        out[n] = _randn(g, (D,), 0.1)
+    if with_weights:
+        out["wqkv"] = _randn(g, (3 * D, D), 0.02)
+        out["wo"] = _randn(g, (D, D), 0.02)
+        out["w1"] = _randn(g, (2 * F, D), 0.02)
+        out["w2"] = _randn(g, (D, F), 0.02)
+    return out
+
+
+def normal_bf16(shape, seed, std=1.0):
+    """A seeded N(0, std^2) bf16 tensor (used for standalone kernel tests)."""
+    g = torch.Generator().manual_seed(seed)
+    return _randn(g, shape, std)
+
+
+def uniform_int(shape, low, high, seed):
+    """Seeded integers in [low, high) as an int64 tensor."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(low, high, shape, generator=g, dtype=torch.int64)
