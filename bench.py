@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Joint-block throughput of the NVFP4 / FP8 FLUX-3-Image-Klein-style joint
+transformer block on B200.
+
+A step is one forward pass of the whole block (LN1+adaLN+NVFP4, QKV GEMM with
+RoPE, FP8 cast, joint attention, NVFP4 of O, output GEMM with gated residual,
+LN2+adaLN+NVFP4, MLP-up GEMM with SwiGLU, NVFP4 of h, MLP-down GEMM with gated
+residual) over one image's token sequence, inputs resident in HBM.  The
+default workload is the 1024x1024 text-to-image block: 512 text + 4,096 image
+tokens (4,608), hidden 3072, 24 heads, MLP 9216, FP8 attention
+(token counts: "Welcome FLUX.3 Image Klein in Diffusers", The VAE and
+Tokenization; "FLUX.3 Image Klein Brings 2-Second AI Image Generation to
+Diffusers", Summary).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle as the reference arm
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own image's
+block (data parallel over images, no collective on the data path): weak
+scaling; timing is the max over ranks of device time.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from synth import MOD_NAMES, WORKLOADS, block_inputs  # noqa: E402
+
+METRIC = "joint-block tokens/s & % of dense FP4/FP8 tensor peak, 1024² T2I and I2I"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+# dense tensor-core ratios to bf16 (nominal B200: bf16 2.25, fp8 4.5, fp4 9 PFLOP/s)
+RATIO = {"fp4": 4.0, "fp8": 2.0, "bf16": 1.0}
+STAGES = ("ln1", "qkv_gemm", "fp8_cast", "attention", "quant_o", "out_gemm", "ln2", "mlp_up_gemm", "quant_h",
+          "mlp_down_gemm")
+KERNELS_PER_STAGE = {"ln1": 2, "qkv_gemm": 1, "fp8_cast": 1, "attention": 1, "quant_o": 1, "out_gemm": 1, "ln2": 2,
+                     "mlp_up_gemm": 1, "quant_h": 1, "mlp_down_gemm": 1}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def stage_work(wl):
+    """Algorithmic work per stage: ("flop", n, dtype) or ("byte", n)."""
+    T, D, H, F = wl.n_tokens, wl.hidden, wl.heads, wl.mlp_hidden
+    nv = 2 + 0.5 + 1 / 16          # bf16 read + NVFP4 codes + scales, bytes per element
+    att_dtype = "fp8" if wl.attn == "fp8" else "bf16"
+    return {
+        "ln1": ("byte", T * D * nv),
+        "qkv_gemm": ("flop", 2.0 * T * 3 * D * D, "fp4"),
+        "fp8_cast": ("byte", T * 3 * D * 3.0),
+        "attention": ("flop", 4.0 * T * T * H * 128, att_dtype),
+        "quant_o": ("byte", T * D * nv),
+        "out_gemm": ("flop", 2.0 * T * D * D, "fp4"),
+        "ln2": ("byte", T * D * nv),
+        "mlp_up_gemm": ("flop", 2.0 * T * 2 * F * D, "fp4"),
+        "quant_h": ("byte", T * F * nv),
+        "mlp_down_gemm": ("flop", 2.0 * T * D * F, "fp4"),
+    }
+
+
+def roofline_entry(work, ms, peaks):
+    if ms <= 0:
+        return None
+    if work[0] == "flop":
+        ach = work[1] / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] * RATIO[work[2]]
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "dtype": work[2]}
+    ach = work[1] / (ms * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": round(peak, 1), "unit": "GB/s",
+            "frac": round(ach / peak, 4)}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = set()
+        for r in rows:
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE {world}")
+    return world, rank, local
+
+
+def config_of(wl, extra=None):
+    c = {"workload": wl.name, "tokens": wl.n_tokens, "text_tokens": wl.n_text,
+         "image_grid": f"{wl.grid_h}x{wl.grid_w}", "reference_images": wl.n_ref, "hidden": wl.hidden,
+         "heads": wl.heads, "head_dim": 128, "mlp_hidden": wl.mlp_hidden, "attention": wl.attn,
+         "weights": "NVFP4 (E2M1, UE4M3 per 16, fp32 global), random N(0,0.02)",
+         "activations": "NVFP4 GEMM inputs, bf16 residual stream N(0,1)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_sample(wl, n_text, grid_rows):
+    """Inputs of a bounded slice of the workload for the CPU oracle: the first
+    n_text text tokens and the first grid_rows rows of the image grid, full
+    widths, the workload's own weights and modulation vectors."""
+    import numpy as np
+
+    from oracle import block, nvfp4
+
+    inp = block_inputs(wl)
+    x = inp["x"].float().numpy()
+    rows = np.concatenate([np.arange(n_text), wl.n_text + np.arange(grid_rows * wl.grid_w)])
+    lay = block.TokenLayout(n_text, grid_rows, wl.grid_w, 0)
+    w = {n: nvfp4.quantize(inp[n].float().numpy()) for n in ("wqkv", "wo", "w1", "w2")}
+    mod = {n: inp[n].float().numpy() for n in MOD_NAMES}
+    return x[rows], mod, w, lay
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, n_text=256, grid_rows=4):
+    from oracle import block
+
+    x, mod, w, lay = oracle_sample(wl, n_text, grid_rows)
+    attn = "fp8" if wl.attn == "fp8" else "exact"
+    t0 = time.perf_counter()
+    block.block_forward(x, mod, w, lay, wl.heads, attn=attn)
+    dt = time.perf_counter() - t0
+    T = lay.n_tokens
+    return {"value": round(T / dt, 3), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{T}-token slice of {wl.name} ({n_text} text + {grid_rows} grid rows x {wl.grid_w}), "
+                      f"full widths, weights pre-encoded (untimed), one block forward: {dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    from oracle import block
+
+    n_text, grid_rows = 64, 1
+    x, mod, w, lay = oracle_sample(wl, n_text, grid_rows)
+    attn = "fp8" if wl.attn == "fp8" else "exact"
+    for _ in range(args.warmup):
+        block.block_forward(x, mod, w, lay, wl.heads, attn=attn)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        block.block_forward(x, mod, w, lay, wl.heads, attn=attn)
+        times.append(time.perf_counter() - t0)
+    T = lay.n_tokens
+    total = sum(times)
+    value = T * args.steps / total
+    sample = (f"each step: {T}-token slice of {wl.name} ({n_text} text + {grid_rows} grid row x {wl.grid_w}), "
+              f"full widths, through the fp64 CPU oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, N(0,0.1) modulation)",
+            "config": config_of(wl, {"sample_tokens": T}),
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------ ours
+def run_ours(args, wl):
+    import diffusion_transformer_image_nvfp4_b200 as kl
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    kl.lib()
+    peaks = load_peaks()
+
+    inp = block_inputs(wl)
+    T, D, H, F = wl.n_tokens, wl.hidden, wl.heads, wl.mlp_hidden
+    d = {k: v.to(dev) for k, v in inp.items()}
+    W = kl.prepare_block_weights(d["wqkv"], d["wo"], d["w1"], d["w2"])
+    cs = kl.rope_table(wl.n_text, wl.grid_h, wl.grid_w, wl.n_ref, device=dev)
+    mod = {n: d[n] for n in MOD_NAMES}
+    x = d["x"]
+    out = torch.empty_like(x)
+    ws = torch.empty(kl.block_workspace_size(T, D, H, F, wl.attn), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    for _ in range(args.warmup):
+        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    st = kl.device_status()
+    if st != "KL_OK":
+        raise SystemExit(f"device status after warm-up: {st}")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        import torch.distributed as dist
+
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    for row in evs:           # materialise the events on this device
+        for e in row:
+            e.record()
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()         # evict L2 between timed steps (outside the events)
+        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws, stage_events=evs[i])
+    barrier()
+    clk = clocks.stop()
+    step_ms = [row[0].elapsed_time(row[-1]) for row in evs]
+    stage_ms = {s: sum(row[j].elapsed_time(row[j + 1]) for row in evs) / args.steps for j, s in enumerate(STAGES)}
+    total_ms = max_over_ranks(sum(step_ms))
+    value = world * T * args.steps / (total_ms * 1e-3)
+
+    # ---- end to end: pinned host x / mod -> device, block, device -> pinned host out
+    x_h = inp["x"].pin_memory()
+    mod_h = {n: inp[n].pin_memory() for n in MOD_NAMES}
+    out_h = torch.empty_like(x_h).pin_memory()
+    x_d = torch.empty_like(x)
+    mod_d = {n: torch.empty_like(mod[n]) for n in MOD_NAMES}
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        x_d.copy_(x_h, non_blocking=True)
+        for n in MOD_NAMES:
+            mod_d[n].copy_(mod_h[n], non_blocking=True)
+        kl.joint_block_forward(W, x_d, mod_d, cs, H, F, attn=wl.attn, out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record()
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev))
+    st = kl.device_status()
+    if st != "KL_OK":
+        raise SystemExit(f"device status after timing: {st}")
+    h2d = T * D * 2 + len(MOD_NAMES) * D * 2
+    d2h = T * D * 2
+
+    work = stage_work(wl)
+    stages = {}
+    for s in STAGES:
+        if wl.attn != "fp8" and s == "fp8_cast":
+            continue
+        ent = roofline_entry(work[s], stage_ms[s], peaks) or {}
+        ent["ms"] = round(stage_ms[s], 4)
+        stages[s] = ent
+    dom = max(stages, key=lambda s: stages[s]["ms"])
+    roof = {k: stages[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac")}
+    roof["kernel"] = dom
+    roof["traffic"] = None
+    roof["peak_source"] = f"{peaks['source']} ({'sustained bf16 x nominal ratio' if roof['bound'] == 'tensor' else 'copy'})"
+    gemm_ms = sum(stage_ms[s] for s in ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm"))
+    gemm_flop = sum(work[s][1] for s in ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm"))
+    fp4_peak = peaks["bf16_tflops_sustained"] * RATIO["fp4"]
+    att_peak = peaks["bf16_tflops_sustained"] * RATIO["fp8" if wl.attn == "fp8" else "bf16"]
+    launches = sum(KERNELS_PER_STAGE[s] for s in stages) * args.steps
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, fp32 acc) + e4m3 attention",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, N(0,0.1) modulation)",
+            "config": config_of(wl, {"parallelism": f"dp{world} (one image per GPU)" if world > 1 else "single GPU",
+                                     "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}),
+            "tflops": round((gemm_flop + work["attention"][1]) / (total_ms / args.steps * 1e-3) / 1e12, 2),
+            "gemm_fp4_frac": round(gemm_flop / (gemm_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "attention_frac": round(work["attention"][1] / (stage_ms["attention"] * 1e-3) / 1e12 / att_peak, 4),
+            "roofline": roof, "stages": stages, "gpu_launches": launches,
+            "e2e": {"value": round(world * T * args.steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="t2i_1024", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

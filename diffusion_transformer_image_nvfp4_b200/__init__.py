@@ -1,0 +1,312 @@
+"""Thin Python binding of libklein.so (the NVFP4 joint-block CUDA library).
+
+Argument marshalling only: every step of the block runs in the library's
+sm_100a kernels.  Tensors are ``torch`` CUDA tensors (PyTorch supplies device
+memory and the current stream); the calls mirror the C ABI in
+``include/klein.h`` and keep its names (``kl_quantize_nvfp4`` ->
+``quantize_nvfp4`` and so on).  There is no CPU or PyTorch fallback: if the
+library is missing every call raises.
+"""
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from .build import LIB_PATH
+
+__all__ = [
+    "KLError", "lib", "NVFP4", "quantize_nvfp4", "ln_modulate_quantize_nvfp4", "gemm_nvfp4_fused",
+    "rope_table", "cast_fp8_per_head", "joint_attention", "BlockWeights", "prepare_block_weights",
+    "joint_block_forward", "block_workspace_size", "device_status", "scales_mma_to_linear",
+]
+
+KL_OK = 0
+STATUS = {0: "KL_OK", 1: "KL_ERR_INVALID_ARG", 2: "KL_ERR_UNSUPPORTED_SHAPE", 3: "KL_ERR_MISALIGNED",
+          4: "KL_ERR_WORKSPACE", 5: "KL_ERR_CUDA", 6: "KL_ERR_DEVICE_TIMEOUT", 7: "KL_ERR_ARCH",
+          8: "KL_ERR_NONFINITE"}
+KL_SCALE_LINEAR, KL_SCALE_MMA, KL_GLOBAL_SCALE_GIVEN, KL_ROWS_SWIGLU_INTERLEAVE = 0, 1, 2, 4
+EPI = {"none": 0, "qkv_rope": 1, "swiglu": 2, "gated_residual": 3}
+KL_OUT_BF16, KL_OUT_F32 = 0, 1
+ATTN = {"fp8": 0, "bf16": 1}
+
+
+class KLError(RuntimeError):
+    def __init__(self, status, where):
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if status == 5 and _LIB is not None:
+            msg += " (" + _LIB.kl_last_cuda_error().decode() + ")"
+        super().__init__(msg)
+        self.status = status
+
+
+class _NVFP4Tensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("global_scale", ctypes.c_void_p)]
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("out_dtype", ctypes.c_int), ("out", ctypes.c_void_p),
+                ("rope_cs", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("amax_out", ctypes.c_void_p)]
+
+
+class _TokenLayout(ctypes.Structure):
+    _fields_ = [("n_text", ctypes.c_int64), ("grid_h", ctypes.c_int64), ("grid_w", ctypes.c_int64),
+                ("n_ref", ctypes.c_int64)]
+
+
+class _BlockWeights(ctypes.Structure):
+    _fields_ = [("wqkv", _NVFP4Tensor), ("wo", _NVFP4Tensor), ("w1", _NVFP4Tensor), ("w2", _NVFP4Tensor)]
+
+
+class _BlockIO(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("mod", ctypes.c_void_p * 6), ("rope_cs", ctypes.c_void_p),
+                ("T", ctypes.c_int64), ("D", ctypes.c_int64), ("H", ctypes.c_int64), ("F", ctypes.c_int64),
+                ("attn_precision", ctypes.c_int), ("out", ctypes.c_void_p),
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+
+
+_LIB = None
+_VP, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "kl_status_string": ([_I], ctypes.c_char_p),
+    "kl_last_cuda_error": ([], ctypes.c_char_p),
+    "kl_version": ([], _I),
+    "kl_device_status": ([_I], _I),
+    "kl_nvfp4_scales_bytes": ([_I64, _I64, _I], _SZ),
+    "kl_quantize_workspace_size": ([], _SZ),
+    "kl_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _I, _VP, _SZ, _VP], _I),
+    "kl_ln_workspace_size": ([_I64], _SZ),
+    "kl_ln_modulate_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
+    "kl_gemm_nvfp4_fused": ([ctypes.POINTER(_NVFP4Tensor), ctypes.POINTER(_NVFP4Tensor), _I64, _I64, _I64,
+                             ctypes.POINTER(_Epilogue), _VP], _I),
+    "kl_layout_tokens": ([ctypes.POINTER(_TokenLayout)], _I64),
+    "kl_rope_table": ([ctypes.POINTER(_TokenLayout), ctypes.c_float, _VP, _VP], _I),
+    "kl_cast_fp8_per_head": ([_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP], _I),
+    "kl_joint_attention_fp8": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _I64, _I64, _I64, _I, _VP, _VP, _VP], _I),
+    "kl_block_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
+    "kl_joint_block_forward": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
+}
+
+
+def lib():
+    """The loaded libklein.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m diffusion_transformer_image_nvfp4_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def _check(status, where):
+    if status != KL_OK:
+        raise KLError(status, where)
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor")
+
+
+_WS = {}
+
+
+def _workspace(nbytes, device, tag):
+    key = (tag, device.index if device.index is not None else torch.cuda.current_device())
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _WS[key] = buf
+    return buf
+
+
+# ---------------------------------------------------------------- NVFP4
+@dataclass
+class NVFP4:
+    """An NVFP4 tensor: codes uint8 [R, C/2]; scales uint8 (linear [R, C/16] or
+    MMA layout, padded to 128-row blocks); gs fp32 [1] decode global scale."""
+
+    codes: torch.Tensor
+    scales: torch.Tensor
+    gs: torch.Tensor
+    rows: int
+    cols: int
+    layout: str
+
+    def abi(self):
+        return _NVFP4Tensor(self.codes.data_ptr(), self.scales.data_ptr(), self.gs.data_ptr())
+
+
+def quantize_nvfp4(x, layout="mma", global_scale=None, swiglu_interleave=False):
+    """kl_quantize_nvfp4 on a contiguous CUDA bf16 [R, C] tensor."""
+    _need(x, torch.bfloat16, "x")
+    R, C = x.shape
+    L = lib()
+    flags = KL_SCALE_MMA if layout == "mma" else KL_SCALE_LINEAR
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, flags & 1), dtype=torch.uint8, device=x.device)
+    if global_scale is not None:
+        flags |= KL_GLOBAL_SCALE_GIVEN
+        gs = torch.as_tensor(global_scale, dtype=torch.float32, device=x.device).reshape(1).clone()
+    else:
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    if swiglu_interleave:
+        flags |= KL_ROWS_SWIGLU_INTERLEAVE
+    ws = _workspace(L.kl_quantize_workspace_size(), x.device, "quant")
+    _check(L.kl_quantize_nvfp4(x.data_ptr(), R, C, codes.data_ptr(), scales.data_ptr(), gs.data_ptr(), flags,
+                               ws.data_ptr(), ws.numel(), _stream()), "kl_quantize_nvfp4")
+    if layout != "mma":
+        scales = scales.view(R, C // 16)
+    return NVFP4(codes, scales, gs, R, C, layout)
+
+
+def ln_modulate_quantize_nvfp4(x, shift, scale, export_m=False):
+    """kl_ln_modulate_quantize_nvfp4: NVFP4 of bf16(LN(x)(1+scale)+shift)."""
+    for t, n in ((x, "x"), (shift, "shift"), (scale, "scale")):
+        _need(t, torch.bfloat16, n)
+    R, C = x.shape
+    L = lib()
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, KL_SCALE_MMA), dtype=torch.uint8, device=x.device)
+    gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    m = torch.empty_like(x) if export_m else None
+    ws = _workspace(L.kl_ln_workspace_size(R), x.device, "ln")
+    _check(L.kl_ln_modulate_quantize_nvfp4(x.data_ptr(), R, C, shift.data_ptr(), scale.data_ptr(), codes.data_ptr(),
+                                           scales.data_ptr(), gs.data_ptr(), _ptr(m), ws.data_ptr(), ws.numel(),
+                                           _stream()), "kl_ln_modulate_quantize_nvfp4")
+    q = NVFP4(codes, scales, gs, R, C, "mma")
+    return (q, m) if export_m else q
+
+
+def gemm_nvfp4_fused(A, W, epilogue="none", out=None, out_dtype=torch.bfloat16, rope_cs=None, gate=None,
+                     residual=None, amax=None):
+    """kl_gemm_nvfp4_fused: C = gA gW dec(A) dec(W)^T with a fused epilogue."""
+    if A.layout != "mma" or W.layout != "mma" or A.cols != W.cols:
+        raise ValueError("operands must share K and use the MMA scale layout")
+    M, N, K = A.rows, W.rows, A.cols
+    kind = EPI[epilogue]
+    if out is None:
+        cols = N // 2 if kind == EPI["swiglu"] else N
+        out = torch.empty((M, cols), dtype=out_dtype, device=A.codes.device)
+    epi = _Epilogue(kind, KL_OUT_F32 if out.dtype == torch.float32 else KL_OUT_BF16, out.data_ptr(), _ptr(rope_cs),
+                    _ptr(gate), _ptr(residual), _ptr(amax))
+    a, w = A.abi(), W.abi()
+    _check(lib().kl_gemm_nvfp4_fused(ctypes.byref(a), ctypes.byref(w), M, N, K, ctypes.byref(epi), _stream()),
+           "kl_gemm_nvfp4_fused")
+    return out
+
+
+def rope_table(n_text, grid_h, grid_w, n_ref=0, theta=10000.0, device="cuda"):
+    """kl_rope_table: fp32 (cos, sin) [T, 64, 2] for the joint sequence."""
+    lay = _TokenLayout(n_text, grid_h, grid_w, n_ref)
+    T = lib().kl_layout_tokens(ctypes.byref(lay))
+    cs = torch.empty((T, 64, 2), dtype=torch.float32, device=device)
+    _check(lib().kl_rope_table(ctypes.byref(lay), theta, cs.data_ptr(), _stream()), "kl_rope_table")
+    return cs
+
+
+def cast_fp8_per_head(x, amax, ncols=None, ld=None):
+    """kl_cast_fp8_per_head: (E4M3 bytes like x, fp32 decode scales [ncols/128])."""
+    T = x.shape[0]
+    ld = x.shape[1] if ld is None else ld
+    ncols = x.shape[1] if ncols is None else ncols
+    out = torch.zeros(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(ncols // 128, dtype=torch.float32, device=x.device)
+    _check(lib().kl_cast_fp8_per_head(x.data_ptr(), T, ncols, ld, amax.data_ptr(), out.data_ptr(), sc.data_ptr(),
+                                      _stream()), "kl_cast_fp8_per_head")
+    return out, sc
+
+
+def joint_attention(q, k, v, T, H, ld, precision="fp8", sq=None, sk=None, sv=None, amax=None, out=None):
+    """kl_joint_attention_fp8 on [T, H, 128] views with row stride ld elements
+    (q, k, v are tensors whose data_ptr is the first element of each)."""
+    if out is None:
+        out = torch.empty((T, H * 128), dtype=torch.bfloat16, device=q.device)
+    _check(lib().kl_joint_attention_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), ld, _ptr(sq), _ptr(sk), _ptr(sv),
+                                        T, H, 128, ATTN[precision], out.data_ptr(), _ptr(amax), _stream()),
+           "kl_joint_attention_fp8")
+    return out
+
+
+# ---------------------------------------------------------------- block
+@dataclass
+class BlockWeights:
+    wqkv: NVFP4
+    wo: NVFP4
+    w1: NVFP4   # SwiGLU-interleaved rows
+    w2: NVFP4
+
+    def abi(self):
+        return _BlockWeights(self.wqkv.abi(), self.wo.abi(), self.w1.abi(), self.w2.abi())
+
+
+def prepare_block_weights(wqkv, wo, w1, w2):
+    """NVFP4-encode bf16 block weights (W1 rows SwiGLU-interleaved) on the GPU."""
+    return BlockWeights(quantize_nvfp4(wqkv), quantize_nvfp4(wo), quantize_nvfp4(w1, swiglu_interleave=True),
+                        quantize_nvfp4(w2))
+
+
+def block_workspace_size(T, D, H, F, attn="fp8"):
+    return lib().kl_block_workspace_size(T, D, H, F, ATTN[attn])
+
+
+BLOCK_STAGES = ("ln1", "qkv_gemm", "fp8_cast", "attention", "quant_o", "out_gemm", "ln2", "mlp_up_gemm",
+                "quant_h", "mlp_down_gemm")
+
+
+def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, workspace=None, stage_events=None):
+    """kl_joint_block_forward.  ``mod`` maps shift1, scale1, gate1, shift2,
+    scale2, gate2 to bf16 [D] CUDA tensors.  ``stage_events`` (optional): a list
+    of len(BLOCK_STAGES)+1 recorded torch.cuda.Event(enable_timing=True); the
+    library re-records them around each stage on the current stream."""
+    _need(x, torch.bfloat16, "x")
+    T, D = x.shape
+    names = ("shift1", "scale1", "gate1", "shift2", "scale2", "gate2")
+    for n in names:
+        _need(mod[n], torch.bfloat16, n)
+    if out is None:
+        out = torch.empty_like(x)
+    need = block_workspace_size(T, D, H, F, attn)
+    if workspace is None:
+        workspace = _workspace(need, x.device, "block")
+    ev = None
+    if stage_events is not None:
+        if len(stage_events) != len(BLOCK_STAGES) + 1:
+            raise ValueError("stage_events: need one event per stage plus one")
+        ev = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+    io = _BlockIO(x.data_ptr(), (ctypes.c_void_p * 6)(*[mod[n].data_ptr() for n in names]), rope_cs.data_ptr(),
+                  T, D, H, F, ATTN[attn], out.data_ptr(), ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)))
+    w = weights.abi()
+    _check(lib().kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(), workspace.numel(),
+                                        _stream()), "kl_joint_block_forward")
+    return out
+
+
+def device_status(clear=True):
+    """kl_device_status: synchronises and returns the status name."""
+    return STATUS.get(lib().kl_device_status(1 if clear else 0), "?")
+
+
+def scales_mma_to_linear(scales, rows, cols):
+    """Reorder a KL_SCALE_MMA scale buffer into the linear [rows, cols/16]
+    layout (index arithmetic of the documented layout; no arithmetic on values)."""
+    r = torch.arange(rows, device=scales.device)[:, None]
+    kb = torch.arange(cols // 16, device=scales.device)[None, :]
+    off = ((r // 128) * (cols // 64) + kb // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + kb % 4
+    return scales.reshape(-1)[off]

@@ -1,0 +1,386 @@
+// kl_gemm.cu -- NVFP4 block-scaled GEMM on 5th-generation tensor cores
+// (tcgen05.mma kind::mxf4nvf4, 16-element UE4M3 block scales), with the fused
+// epilogues of the joint block: RoPE + per-head amax on the QKV projection,
+// SwiGLU + amax on the MLP up projection, adaLN-gated residual on the output
+// and MLP down projections.
+//
+// [P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs",
+// How it works: NVFP4 weights and activations feed optimised GEMM kernels that
+// fuse SwiGLU activations and rotary position embeddings.  The page names
+// those kernels (PrimsTS) but gives no design; this one is written for B200:
+//
+//  * persistent grid (one 192-thread CTA per SM), 128 x BN output tiles,
+//    BN = 256 (one TMEM accumulator) or 128 (two, so the epilogue of tile i
+//    overlaps the main loop of tile i+1);
+//  * warp 0 lane 0: TMA producer.  A [128 x 256] and W [BN x 256] FP4 tiles
+//    (128 bytes per row, 128-byte swizzle) by cp.async.bulk.tensor; the block
+//    scales for those tiles, already stored in the MMA scale layout, by
+//    cp.async.bulk (contiguous 512-byte atoms);
+//  * warp 1 lane 0: MMA issuer.  Per 64-wide K step: tcgen05.cp of the A and
+//    W scale atoms into TMEM, then one 128 x BN x 64 block-scaled MMA into the
+//    TMEM accumulator; tcgen05.commit releases smem stages / publishes tiles;
+//  * warps 2-5: epilogue.  tcgen05.ld 32 columns at a time (thread = row),
+//    scale by gA*gW, apply the fused epilogue, store bf16/fp32.
+// Smem ring: 4 (BN 256) or 6 (BN 128) stages of ~54 / 36 KB.
+#include "kl_common.cuh"
+#include "kl_internal.h"
+#include "../../include/klein.h"
+
+namespace kl {
+
+struct GemmParams {
+  int64_t M, N, K;
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* gsa;
+  const float* gsw;
+  int epi, out_f32;
+  void* out;
+  const float2* rope_cs;
+  const uint16_t* gate;
+  const uint16_t* residual;
+  float* amax;
+  int num_m, num_tiles, num_kt, kbn;  // kbn = K / 64
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFA_BYTES = 2048;
+  static constexpr int SFB_BYTES = (BN / 128) * 2048;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int ACC = BN == 256 ? 1 : 2;
+  static constexpr uint32_t SFA_COL = ACC * BN;
+  static constexpr uint32_t SFB_COL = SFA_COL + 16;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(SFB_COL + 4 * (BN / 32) <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "smem budget");
+};
+
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+__device__ __forceinline__ void load_bf16x32(const uint16_t* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w = __ldg(s + q);
+    uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * q + 2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
+      v[8 * q + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+    }
+  }
+}
+// round to bf16 in place (the stored value), returning max |.|
+__device__ __forceinline__ float round_bf16x32(float (&v)[32]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = bf16_bits_to_f32(f32_to_bf16_bits(v[i]));
+    m = fmaxf(m, fabsf(v[i]));
+  }
+  return m;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const GemmParams p) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + C::ACC;
+  uint64_t* drain = tempty + C::ACC;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < C::ACC; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          uint8_t* ssfa = sb + C::B_BYTES;
+          uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          const int nk = min(4, p.kbn - kt * 4);
+          const uint32_t sf_bytes = (uint32_t)nk * 512u;
+          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
+          tma_load_2d(sa, &tmap_a, kt * 128, mb * 128, &full[stage]);
+          tma_load_2d(sb, &tmap_b, kt * 128, nb * BN, &full[stage]);
+          bulk_load(ssfa, p.sfa + ((int64_t)mb * p.kbn + kt * 4) * 512, sf_bytes, &full[stage]);
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j)
+            bulk_load(ssfb + j * 2048, p.sfb + ((int64_t)(nb * (BN / 128) + j) * p.kbn + kt * 4) * 512, sf_bytes,
+                      &full[stage]);
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every load already issued land before the CTA can exit
+        const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
+        for (int64_t i = first; i < issued; ++i) {
+          volatile int no_abort = 0;
+          mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), &no_abort);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_nvf4(128, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          const uint8_t* sb = sa + C::A_BYTES;
+          const uint8_t* ssfa = sb + C::B_BYTES;
+          const uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          const int nk = min(4, p.kbn - kt * 4);
+          for (int kk = 0; kk < nk; ++kk) {
+            tmem_cp_32x128b_x4(tmem + C::SFA_COL + kk * 4, smem_desc(smem_u32(ssfa + kk * 512), 0, 128, kLayoutNone));
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tmem_cp_32x128b_x4(tmem + C::SFB_COL + kk * (BN / 32) + j * 4,
+                                 smem_desc(smem_u32(ssfb + j * 2048 + kk * 512), 0, 128, kLayoutNone));
+          }
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = smem_desc(smem_u32(sa + kk * 32), 16, 1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(smem_u32(sb + kk * 32), 16, 1024, kLayoutSw128);
+            mma_nvf4(d_tmem, ad, bd, idesc, tmem + C::SFA_COL + kk * 4, tmem + C::SFB_COL + kk * (BN / 32),
+                     (kt | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        if (++acc == C::ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // every MMA / copy issued by this thread has completed before TMEM is freed
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    const float alpha = __fmul_rn(__ldg(p.gsa), __ldg(p.gsw));
+    const int64_t D = p.N / 3;           // QKV only
+    const int H = (int)(D >> 7);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int64_t row = (int64_t)mb * 128 + row_in_tile;
+      const bool valid = row < p.M;
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      const int64_t n0 = (int64_t)nb * BN;
+      if (p.epi == KL_EPI_SWIGLU) {
+        float amax = 0.f;
+        const int64_t F = p.N >> 1;
+#pragma unroll 1
+        for (int g = 0; g < BN / 128; ++g) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            float vg[32], vu[32];
+            tmem_ld32(tbase + g * 128 + c0, vg);
+            tmem_ld32(tbase + g * 128 + 64 + c0, vu);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float gg = vg[i] * alpha, uu = vu[i] * alpha;
+              vg[i] = gg / (1.0f + expf(-gg)) * uu;
+            }
+            amax = fmaxf(amax, round_bf16x32(vg));
+            if (valid)
+              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + g * 64 + c0, vg);
+          }
+        }
+        amax = warp_max(valid ? amax : 0.f);
+        if (lane == 0) atomic_max_nonneg(p.amax, amax);
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float v[32];
+          tmem_ld32(tbase + c0, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          const int64_t n = n0 + c0;
+          if (p.epi == KL_EPI_NONE) {
+            if (valid) {
+              if (p.out_f32) {
+                float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.N + n);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              } else {
+                store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+              }
+            }
+          } else if (p.epi == KL_EPI_GATED_RESIDUAL) {
+            float gt[32], rs[32];
+            load_bf16x32(p.gate + n, gt);
+            if (valid) {
+              load_bf16x32(p.residual + row * p.N + n, rs);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = __fmaf_rn(gt[i], v[i], rs[i]);
+              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+            }
+          } else {  // KL_EPI_QKV_ROPE
+            const int region = (int)(n / D);
+            const int64_t cc = n - (int64_t)region * D;
+            const int head = (int)(cc >> 7);
+            if (region < 2) {
+              const int j0 = (int)((cc & 127) >> 1);
+              const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (valid ? row : 0) * 64 + j0);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 t = __ldg(cs + q);  // (c, s) of two consecutive pairs
+                const float a0 = v[4 * q], b0 = v[4 * q + 1], a1 = v[4 * q + 2], b1 = v[4 * q + 3];
+                v[4 * q] = a0 * t.x - b0 * t.y;
+                v[4 * q + 1] = a0 * t.y + b0 * t.x;
+                v[4 * q + 2] = a1 * t.z - b1 * t.w;
+                v[4 * q + 3] = a1 * t.w + b1 * t.z;
+              }
+            }
+            float amax = round_bf16x32(v);
+            if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+            amax = warp_max(valid ? amax : 0.f);
+            if (lane == 0) atomic_max_nonneg(p.amax + region * H + head, amax);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == C::ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN>
+static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
+                    (uint64_t)(a.K / 2), 128, 128))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                    (uint64_t)(a.K / 2), 128, BN))
+    return cudaErrorInvalidValue;
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.sfa = reinterpret_cast<const uint8_t*>(a.a_scales);
+  p.sfb = reinterpret_cast<const uint8_t*>(a.w_scales);
+  p.gsa = a.a_gs;
+  p.gsw = a.w_gs;
+  p.epi = a.epi;
+  p.out_f32 = a.out_f32;
+  p.out = a.out;
+  p.rope_cs = reinterpret_cast<const float2*>(a.rope_cs);
+  p.gate = reinterpret_cast<const uint16_t*>(a.gate);
+  p.residual = reinterpret_cast<const uint16_t*>(a.residual);
+  p.amax = a.amax;
+  p.num_m = (int)((a.M + 127) / 128);
+  p.num_tiles = p.num_m * (int)(a.N / BN);
+  p.kbn = (int)(a.K / 64);
+  p.num_kt = (p.kbn + 3) / 4;
+  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
+  gemm_nvfp4_kernel<BN><<<grid, 192, C::SMEM_BYTES, s>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
+  int bn = a.force_bn;
+  if (bn == 0) bn = (a.N % 256 == 0) ? 256 : 128;
+  if (bn == 256 && a.N % 256 != 0) return cudaErrorInvalidValue;
+  return bn == 256 ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
+}
+
+}  // namespace kl

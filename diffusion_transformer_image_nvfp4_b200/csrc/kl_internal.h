@@ -1,0 +1,66 @@
+// kl_internal.h -- host-side launchers shared by the libklein translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kl {
+
+constexpr int kNumSMs = 148;  // B200; only caps grid-stride grids (persistent kernels query the device)
+
+int device_sm_count();  // cached per process
+
+// HBM-bound kernels (kl_quant.cu)
+cudaError_t launch_amax_bf16(const void* x, int64_t n, float* amax, cudaStream_t s);
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols, void* codes, void* scales, float* gs_io,
+                            const float* amax, int mode, cudaStream_t s);
+cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t cols, const void* shift,
+                                        const void* scale, void* codes, void* scales, float* gs_out,
+                                        void* m_out, float2* stats, float* amax, cudaStream_t s);
+cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
+                            float* scales_out, cudaStream_t s);
+cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,
+                              cudaStream_t s);
+
+// tcgen05 NVFP4 GEMM (kl_gemm.cu)
+struct GemmArgs {
+  const void* a_codes;
+  const void* a_scales;
+  const float* a_gs;
+  const void* w_codes;
+  const void* w_scales;
+  const float* w_gs;
+  int64_t M, N, K;
+  int epi;        // KL_EPI_*
+  int out_f32;    // KL_EPI_NONE only
+  void* out;
+  const float* rope_cs;
+  const void* gate;
+  const void* residual;
+  float* amax;
+  int force_bn;   // 0 = heuristic, else 128 or 256
+};
+cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s);
+
+// tcgen05 flash attention (kl_attn.cu)
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t ld;  // row stride in elements
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  int64_t T, H;
+  int fp8;
+  void* out;   // bf16 [T, H*128]
+  float* amax; // nullable
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// tensor maps (kl_api.cu)
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace kl

@@ -1,0 +1,349 @@
+// kl_quant.cu -- the HBM-bound kernels of the block: per-tensor amax, the
+// NVFP4 quantiser, fused LayerNorm + adaLN modulation + NVFP4 quantiser, the
+// per-head FP8 cast of Q/K/V, and the RoPE cos/sin table.
+//
+// NVFP4 reading (the NVFP4 variant of "Optimizing FLUX 3 Image Klein inference
+// on NVIDIA Blackwell GPUs", How it works; the page names the format but not
+// its encoding): E2M1 codes, one unsigned E4M3 scale per 16 elements, fp32
+// decode global scale gs = amax/2688.  Every step is one IEEE fp32 operation
+// with round-to-nearest-even (explicit __f*_rn intrinsics, so no FMA
+// contraction and no approximate reciprocal can change a code), then the
+// hardware cvt.rn.satfinite conversions to E4M3 / E2M1.
+#include "kl_common.cuh"
+#include "kl_internal.h"
+
+namespace kl {
+
+constexpr float kGsDivisor = 2688.0f;  // 6 * 448
+
+// ------------------------------------------------------------------ amax
+// max |x| over n bf16 values (n % 8 == 0, 16-byte aligned) into *amax (which
+// the launcher zeroes first).  Non-finite input sets KL_DEVERR_NONFINITE.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict__ x, int64_t n8,
+                                                        float* __restrict__ amax) {
+  float m = 0.f;
+  bool bad = false;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    uint4 v = __ldg(x + i);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+      bad |= (lo >= 0x7F80u) | (hi >= 0x7F80u);
+      m = fmaxf(m, fmaxf(__uint_as_float(lo << 16), __uint_as_float(hi << 16)));
+    }
+  }
+  m = warp_max(m);
+  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = m;
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(KL_DEVERR_NONFINITE);
+  __syncthreads();
+  if (warp == 0) {
+    m = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    m = warp_max(m);
+    if (lane == 0) atomic_max_nonneg(amax, m);
+  }
+}
+
+// --------------------------------------------------------- block encoder
+struct GsParams {
+  float gs, inv;  // decode global scale and 1/(6 gs)
+};
+__device__ __forceinline__ GsParams gs_from_amax(float amax) {
+  GsParams p;
+  p.gs = amax == 0.f ? 1.0f : __fdiv_rn(amax, kGsDivisor);
+  p.inv = __fdiv_rn(1.0f, __fmul_rn(6.0f, p.gs));
+  return p;
+}
+__device__ __forceinline__ GsParams gs_given(float gs) {
+  GsParams p;
+  p.gs = gs;
+  p.inv = __fdiv_rn(1.0f, __fmul_rn(6.0f, gs));
+  return p;
+}
+
+// Encode 16 values: returns the scale byte, writes 8 packed code bytes.
+__device__ __forceinline__ uint32_t encode_block16(const float (&v)[16], const GsParams& g, uint2& packed) {
+  float amax_b = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+  uint32_t sb = amax_b > 0.f ? f32_to_e4m3(__fmul_rn(amax_b, g.inv)) : 0u;
+  const float S = __fmul_rn(e4m3_to_f32(sb), g.gs);
+  if (S == 0.f) {
+    packed = make_uint2(0u, 0u);
+    return sb;
+  }
+  const float r = __fdiv_rn(1.0f, S);
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(v[i], r);
+  packed.x = f32x8_to_e2m1x8(y);
+  packed.y = f32x8_to_e2m1x8(y + 8);
+  return sb;
+}
+
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t row, int64_t kb, int64_t cols) {
+  const int64_t rb = row >> 7, r = row & 127;
+  return ((rb * (cols >> 6) + (kb >> 2)) << 9) + ((r & 31) << 4) + ((r >> 5) << 2) + (kb & 3);
+}
+
+__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&v)[16]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+    v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+  }
+}
+
+__device__ __forceinline__ int64_t swiglu_src_row(int64_t r, int64_t rows) {
+  const int64_t g = r >> 7, i = r & 127;
+  return i < 64 ? (g << 6) + i : (rows >> 1) + (g << 6) + (i - 64);
+}
+
+// One thread per 16-element block.  mode bits: 1 = MMA scale layout,
+// 2 = gs given (read *gs_io), 4 = SwiGLU row interleave.
+__global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                       int64_t cols, int64_t rows_padded,
+                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                       float* __restrict__ gs_io, const float* __restrict__ amax,
+                                                       int mode) {
+  const bool mma = mode & 1, given = mode & 2, perm = mode & 4;
+  const GsParams g = given ? gs_given(*gs_io) : gs_from_amax(*amax);
+  const int64_t kbn = cols >> 4;
+  const int64_t total = rows_padded * kbn;
+  if (!given && blockIdx.x == 0 && threadIdx.x == 0) *gs_io = g.gs;
+  for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < total; b += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = b / kbn, kb = b - row * kbn;
+    const int64_t soff = mma ? mma_scale_offset(row, kb, cols) : row * kbn + kb;
+    if (row >= rows) {  // padding rows of the MMA layout
+      scales[soff] = 0;
+      continue;
+    }
+    const int64_t src = perm ? swiglu_src_row(row, rows) : row;
+    float v[16];
+    load16_bf16(x + src * cols + (kb << 4), v);
+    uint2 pk;
+    const uint32_t sb = encode_block16(v, g, pk);
+    *reinterpret_cast<uint2*>(codes + row * (cols >> 1) + (kb << 3)) = pk;
+    scales[soff] = (uint8_t)sb;
+  }
+}
+
+// ---------------------------------------------- LayerNorm + adaLN modulate
+// m = bf16( ((x - mean) * rstd) * (1 + scale) + shift ), each step rounded.
+__device__ __forceinline__ float ln_mod_value(float xv, float mean, float rstd, float onep, float shift) {
+  const float y = __fmul_rn(__fsub_rn(xv, mean), rstd);
+  return bf16_bits_to_f32(f32_to_bf16_bits(__fmaf_rn(y, onep, shift)));
+}
+
+// One warp per row: mean and rstd (fp32, two passes), then amax of m.
+__global__ void __launch_bounds__(256) ln_stats_amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                            int64_t cols, const uint16_t* __restrict__ shift,
+                                                            const uint16_t* __restrict__ scale,
+                                                            float2* __restrict__ stats, float* __restrict__ amax) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + warp;
+  float m = 0.f;
+  if (row < rows) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+    const int n8 = (int)(cols >> 3);
+    float s = 0.f;
+    for (int i = lane; i < n8; i += 32) {
+      uint4 v = __ldg(xr + i);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s += bf16_bits_to_f32(w[j] & 0xFFFFu) + bf16_bits_to_f32(w[j] >> 16);
+    }
+    const float mean = __fdiv_rn(warp_sum(s), (float)cols);
+    float ss = 0.f;
+    for (int i = lane; i < n8; i += 32) {
+      uint4 v = __ldg(xr + i);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float a = bf16_bits_to_f32(w[j] & 0xFFFFu) - mean, b = bf16_bits_to_f32(w[j] >> 16) - mean;
+        ss += a * a + b * b;
+      }
+    }
+    const float var = __fdiv_rn(warp_sum(ss), (float)cols);
+    const float rstd = __frsqrt_rn(__fadd_rn(var, 1e-6f));
+    if (lane == 0) stats[row] = make_float2(mean, rstd);
+    const uint4* shr = reinterpret_cast<const uint4*>(shift);
+    const uint4* scr = reinterpret_cast<const uint4*>(scale);
+    for (int i = lane; i < n8; i += 32) {
+      uint4 v = __ldg(xr + i), sh = __ldg(shr + i), sc = __ldg(scr + i);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w}, a[4] = {sh.x, sh.y, sh.z, sh.w}, c[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t sft = h ? 16 : 0;
+          const float xv = bf16_bits_to_f32((w[j] >> sft) & 0xFFFFu);
+          const float onep = __fadd_rn(1.0f, bf16_bits_to_f32((c[j] >> sft) & 0xFFFFu));
+          const float mv = ln_mod_value(xv, mean, rstd, onep, bf16_bits_to_f32((a[j] >> sft) & 0xFFFFu));
+          m = fmaxf(m, fabsf(mv));
+        }
+      }
+    }
+  }
+  m = warp_max(m);
+  if (lane == 0 && row < rows) atomic_max_nonneg(amax, m);
+}
+
+// One thread per 16-element block: recompute m and encode it (MMA layout).
+__global__ void __launch_bounds__(256) ln_quant_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                                                       int64_t rows_padded, const uint16_t* __restrict__ shift,
+                                                       const uint16_t* __restrict__ scale,
+                                                       const float2* __restrict__ stats,
+                                                       const float* __restrict__ amax, uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ scales, float* __restrict__ gs_out,
+                                                       uint16_t* __restrict__ m_out) {
+  const GsParams g = gs_from_amax(*amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = g.gs;
+  const int64_t kbn = cols >> 4;
+  const int64_t total = rows_padded * kbn;
+  for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < total; b += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = b / kbn, kb = b - row * kbn;
+    const int64_t soff = mma_scale_offset(row, kb, cols);
+    if (row >= rows) {
+      scales[soff] = 0;
+      continue;
+    }
+    const float2 st = stats[row];
+    float xv[16], sh[16], sc[16], v[16];
+    load16_bf16(x + row * cols + (kb << 4), xv);
+    load16_bf16(shift + (kb << 4), sh);
+    load16_bf16(scale + (kb << 4), sc);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = ln_mod_value(xv[i], st.x, st.y, __fadd_rn(1.0f, sc[i]), sh[i]);
+    if (m_out) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+      uint4* dst = reinterpret_cast<uint4*>(m_out + row * cols + (kb << 4));
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    uint2 pk;
+    const uint32_t sb = encode_block16(v, g, pk);
+    *reinterpret_cast<uint2*>(codes + row * (cols >> 1) + (kb << 3)) = pk;
+    scales[soff] = (uint8_t)sb;
+  }
+}
+
+// ------------------------------------------------------------ FP8 cast
+// 16 elements per thread (inside one 128-wide head).
+__global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t ncols,
+                                                       int64_t ld, const float* __restrict__ amax,
+                                                       uint8_t* __restrict__ out, float* __restrict__ scales_out) {
+  const int64_t n16 = ncols >> 4;
+  const int64_t total = T * n16;
+  const int64_t nheads = ncols >> 7;
+  if (blockIdx.x == 0 && threadIdx.x < nheads) {
+    const float a = amax[threadIdx.x];
+    scales_out[threadIdx.x] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
+  }
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / n16, c = (i - t * n16) << 4;
+    const float a = __ldg(amax + (c >> 7));
+    const float inv = a > 0.f ? __fdiv_rn(448.0f, a) : 1.0f;
+    float v[16];
+    load16_bf16(x + t * ld + c, v);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = f32x2_to_e4m3x2(__fmul_rn(v[4 * j], inv), __fmul_rn(v[4 * j + 1], inv)) |
+             (f32x2_to_e4m3x2(__fmul_rn(v[4 * j + 2], inv), __fmul_rn(v[4 * j + 3], inv)) << 16);
+    *reinterpret_cast<uint4*>(out + t * ld + c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ------------------------------------------------------------ RoPE table
+__global__ void rope_table_kernel(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta,
+                                  float2* __restrict__ cs) {
+  const int64_t T = n_text + (1 + n_ref) * gh * gw;
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= T * 64) return;
+  const int64_t t = i >> 6;
+  const int j = (int)(i & 63);
+  double phi;
+  if (t < n_text) {
+    phi = (double)t * pow(theta, -2.0 * j / 128.0);
+  } else {
+    const int64_t s = t - n_text, img = gh * gw;
+    const int64_t f = s / img, rc = s - f * img, r = rc / gw, c = rc - r * gw;
+    if (j < 16)
+      phi = (double)f * pow(theta, -2.0 * j / 32.0);
+    else if (j < 40)
+      phi = (double)r * pow(theta, -2.0 * (j - 16) / 48.0);
+    else
+      phi = (double)c * pow(theta, -2.0 * (j - 40) / 48.0);
+  }
+  cs[i] = make_float2((float)cos(phi), (float)sin(phi));
+}
+
+// --------------------------------------------------------------- launchers
+static int grid_for(int64_t work, int threads) {
+  int64_t g = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)kNumSMs * 16;
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_amax_bf16(const void* x, int64_t n, float* amax, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  amax_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), n / 8, amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols, void* codes, void* scales, float* gs_io,
+                            const float* amax, int mode, cudaStream_t s) {
+  const int64_t rows_padded = (mode & 1) ? ((rows + 127) / 128) * 128 : rows;
+  quantize_kernel<<<grid_for(rows_padded * (cols / 16), 256), 256, 0, s>>>(
+      reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<uint8_t*>(codes),
+      reinterpret_cast<uint8_t*>(scales), gs_io, amax, mode);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t cols, const void* shift,
+                                        const void* scale, void* codes, void* scales, float* gs_out,
+                                        void* m_out, float2* stats, float* amax, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (rows + 7) / 8;
+  ln_stats_amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), rows, cols,
+                                                        reinterpret_cast<const uint16_t*>(shift),
+                                                        reinterpret_cast<const uint16_t*>(scale), stats, amax);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t rows_padded = ((rows + 127) / 128) * 128;
+  ln_quant_kernel<<<grid_for(rows_padded * (cols / 16), 256), 256, 0, s>>>(
+      reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<const uint16_t*>(shift),
+      reinterpret_cast<const uint16_t*>(scale), stats, amax, reinterpret_cast<uint8_t*>(codes),
+      reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
+                            float* scales_out, cudaStream_t s) {
+  fp8_cast_kernel<<<grid_for(T * (ncols / 16), 256), 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), T, ncols,
+                                                                  ld, amax, reinterpret_cast<uint8_t*>(out),
+                                                                  scales_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,
+                              cudaStream_t s) {
+  const int64_t T = n_text + (1 + n_ref) * gh * gw;
+  const int64_t n = T * 64;
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(n_text, gh, gw, n_ref, theta,
+                                                               reinterpret_cast<float2*>(cs));
+  return cudaGetLastError();
+}
+
+}  // namespace kl

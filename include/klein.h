@@ -1,0 +1,297 @@
+/*
+ * klein.h -- C ABI of libklein.so: the forward pass of one FLUX-3-Image-Klein-
+ * style joint transformer block on NVIDIA B200 (sm_100a), built from NVFP4
+ * block-scaled GEMMs (tcgen05, TMEM accumulators) with fused RoPE / SwiGLU /
+ * gated-residual epilogues and a flash-style FP8 (or BF16) joint attention.
+ *
+ * Sources (page titles and sections):
+ *  [P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs",
+ *       How it works: NVFP4 weights and activations; GEMM kernels that fuse
+ *       SwiGLU and rotary position embeddings; FP8 query/key/value attention.
+ *  [P2] "FLUX.3 Image Klein Brings 2-Second AI Image Generation to Diffusers",
+ *       Summary: 28 joint transformer blocks merge text, generated-image and
+ *       reference tokens; a 1024x1024 reference adds 4,096 tokens.
+ *  [P4] "Welcome FLUX.3 Image Klein in Diffusers", Architecture and Technical
+ *       Deep Dive: 64x64 = 4,096 tokens per 1024x1024 image; 3072-wide
+ *       transformer; joint blocks attend over the concatenated streams.
+ * The pages do not define the NVFP4 encoding or the block's wiring; the
+ * readings implemented here are stated at each entry point.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  Nothing on
+ *    this path allocates or frees device memory; scratch comes from a caller
+ *    workspace whose size a *_workspace_size call returns.
+ *  - Every call is asynchronous on the given CUDA stream (cudaStream_t passed
+ *    as void*; NULL = legacy default stream) and returns a kl_status.  Host-side
+ *    argument checks return an error before anything is enqueued.  Device-side
+ *    conditions (a bounded wait that expired, a non-finite input) are recorded
+ *    in a per-device status word that kl_device_status() reads.
+ *  - Shapes are int64_t, row-major, rows x columns.  bf16 tensors are passed
+ *    as uint16_t bit patterns.  Pointers must be 16-byte aligned (128-byte
+ *    aligned for operands read by TMA: NVFP4 codes, FP8/bf16 Q/K/V).
+ *  - No C++ exception crosses this ABI.
+ */
+#ifndef KLEIN_H
+#define KLEIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int kl_status;
+#define KL_OK 0
+#define KL_ERR_INVALID_ARG 1       /* null pointer, bad enum, bad stride */
+#define KL_ERR_UNSUPPORTED_SHAPE 2 /* a dimension this library does not tile */
+#define KL_ERR_MISALIGNED 3        /* pointer alignment rule broken */
+#define KL_ERR_WORKSPACE 4         /* workspace missing or too small */
+#define KL_ERR_CUDA 5              /* a CUDA runtime/driver call failed */
+#define KL_ERR_DEVICE_TIMEOUT 6    /* a bounded device wait expired (device status) */
+#define KL_ERR_ARCH 7              /* current device is not sm_100 */
+#define KL_ERR_NONFINITE 8         /* NaN/Inf met by an amax pass (device status) */
+
+/* Human-readable name of a status code (static string). */
+const char* kl_status_string(kl_status s);
+/* Text of the last CUDA error seen by this library on this thread ("" if none). */
+const char* kl_last_cuda_error(void);
+/* Library version, major*10000 + minor*100 + patch. */
+int kl_version(void);
+
+/*
+ * Device status word of the current device.  Synchronises the device, then
+ * returns KL_OK, KL_ERR_DEVICE_TIMEOUT or KL_ERR_NONFINITE (the first recorded
+ * condition, timeouts first).  If `clear` is non-zero the word is reset to 0.
+ * Kernels never trap: an expired wait sets the word and the kernel returns.
+ */
+kl_status kl_device_status(int clear);
+
+/* ------------------------------------------------------------------------
+ * NVFP4 tensors
+ *
+ * Reading of NVFP4 ([P1] How it works names the format, not the encoding):
+ * E2M1 element codes, one unsigned E4M3 decode scale per 16 consecutive
+ * elements of a row, one fp32 per-tensor decode scale gs; decoded value =
+ * e2m1(code) * e4m3(scale) * gs.  Codes: uint8 [R, C/2], element 2i in the
+ * low nibble of byte i.  Scales ("scale layouts"):
+ *   KL_SCALE_LINEAR : uint8 [R, C/16] row-major;
+ *   KL_SCALE_MMA    : the tcgen05 block-scale layout, padded to
+ *                     ceil(R/128)*128 rows: 512-byte atoms, one per
+ *                     (128-row block rb, 64-column block kb), atom index
+ *                     rb*(C/64) + kb, byte (r%32)*16 + ((r/32)%4)*4 + (c/16)%4
+ *                     inside the atom.  Padding rows hold scale 0.
+ * ---------------------------------------------------------------------- */
+#define KL_SCALE_LINEAR 0
+#define KL_SCALE_MMA 1
+#define KL_GLOBAL_SCALE_GIVEN 2    /* use *global_scale as gs instead of amax/2688 */
+#define KL_ROWS_SWIGLU_INTERLEAVE 4/* output row r reads input row perm(r), see below */
+
+/* Bytes of the scale array for an [R, C] NVFP4 tensor in the given layout. */
+size_t kl_nvfp4_scales_bytes(int64_t rows, int64_t cols, int layout);
+
+/* Workspace bytes kl_quantize_nvfp4 needs (an amax word). */
+size_t kl_quantize_workspace_size(void);
+
+/*
+ * kl_quantize_nvfp4 -- NVFP4-encode a bf16 tensor x [rows, cols].
+ * cols % 16 == 0 (% 64 for KL_SCALE_MMA).  Steps, each an IEEE fp32 operation
+ * rounded to nearest even: amax_t = max|x|; gs = amax_t/2688 (1 if amax_t==0)
+ * unless KL_GLOBAL_SCALE_GIVEN; inv = 1/(6*gs); per 16-block
+ * sb = e4m3_rne_satfinite(amax_b*inv) (0 if amax_b==0); S = e4m3(sb)*gs;
+ * code_i = e2m1_rne_satfinite(x_i * (1/S)) (all 0 if S==0).
+ * Output: codes [rows, cols/2]; scales (layout from flags); *global_scale = gs
+ * (device fp32; read instead of written with KL_GLOBAL_SCALE_GIVEN).
+ * KL_ROWS_SWIGLU_INTERLEAVE (rows % 128 == 0): output row r holds input row
+ *   (r/128)*64 + (r%128)       if r%128 < 64   (gate half, rows [0, rows/2))
+ *   rows/2 + (r/128)*64 + r%64 otherwise        (up half, rows [rows/2, rows))
+ * i.e. each 128-row group is 64 gate rows followed by the matching 64 up rows,
+ * the layout the SwiGLU GEMM epilogue expects for W1.
+ * workspace: >= kl_quantize_workspace_size() bytes, 16-byte aligned.
+ * Non-finite input is undefined; the amax pass records KL_ERR_NONFINITE.
+ */
+kl_status kl_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t cols,
+                            void* codes, void* scales, float* global_scale, int flags,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kl_ln_modulate_quantize_nvfp4 -- fused LayerNorm + adaLN modulation +
+ * NVFP4 encode of x [rows, cols] bf16 (the pre-attention and pre-MLP step of
+ * the block).  Reading ([P1]/[P2] do not define the wiring): LN over cols
+ * with biased variance and eps 1e-6, no affine;
+ * m = bf16(LN(x) * (1 + scale) + shift) with shift/scale bf16 [cols] shared by
+ * all rows; then the kl_quantize_nvfp4 encoding of m (dynamic gs from amax of
+ * m, scales in KL_SCALE_MMA layout).  m_out (nullable) receives m as bf16
+ * [rows, cols] (a debug export).  cols % 64 == 0, cols <= 8192.
+ * workspace: >= kl_ln_workspace_size(rows).
+ */
+size_t kl_ln_workspace_size(int64_t rows);
+kl_status kl_ln_modulate_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t cols,
+                                        const void* shift_bf16, const void* scale_bf16,
+                                        void* codes, void* scales, float* global_scale,
+                                        void* m_out_bf16, void* workspace, size_t ws_bytes,
+                                        void* stream);
+
+/* An NVFP4 GEMM operand: codes [R, K/2], scales in KL_SCALE_MMA layout,
+ * global decode scale (device fp32). */
+typedef struct kl_nvfp4_tensor {
+  const void* codes;
+  const void* scales;
+  const float* global_scale;
+} kl_nvfp4_tensor;
+
+/* GEMM epilogues */
+#define KL_EPI_NONE 0            /* out[m,n] = acc (bf16 or fp32)                   */
+#define KL_EPI_QKV_ROPE 1        /* q|k|v split, RoPE on q and k, per-head amax     */
+#define KL_EPI_SWIGLU 2          /* h = silu(gate)*up over interleaved rows, amax   */
+#define KL_EPI_GATED_RESIDUAL 3  /* out = residual + gate[n] * acc                  */
+
+#define KL_OUT_BF16 0
+#define KL_OUT_F32 1
+
+typedef struct kl_epilogue {
+  int kind;               /* KL_EPI_* */
+  int out_dtype;          /* KL_OUT_BF16 (all kinds) or KL_OUT_F32 (KL_EPI_NONE only) */
+  void* out;              /* NONE/GATED_RESIDUAL/QKV_ROPE: [M, N]; SWIGLU: [M, N/2]; row-major */
+  const float* rope_cs;   /* QKV_ROPE: fp32 [M, 64, 2] (cos, sin) per token and pair */
+  const void* gate;       /* GATED_RESIDUAL: bf16 [N] */
+  const void* residual;   /* GATED_RESIDUAL: bf16 [M, N] (may alias nothing else written) */
+  float* amax_out;        /* QKV_ROPE: [3*N/384] per (q|k|v, head) max|out|; SWIGLU: [1].
+                             Max-accumulated as non-negative floats: caller zero-fills. */
+} kl_epilogue;
+
+/*
+ * kl_gemm_nvfp4_fused -- C[M,N] = gA*gW * sum_k dec(A)[m,k] * dec(W)[n,k]
+ * (both operands K-major, "y = x W^T") on tcgen05 block-scaled FP4 tensor
+ * cores, followed by the epilogue:
+ *  NONE           out = C.
+ *  QKV_ROPE       N = 3*D, D = 128*H.  Columns [0,D) are q, [D,2D) k, [2D,3D)
+ *                 v; head h = columns [128h, 128h+128) of each.  q and k pairs
+ *                 (2j, 2j+1) are rotated (a,b) -> (a c - b s, a s + b c) with
+ *                 (c, s) = rope_cs[m, j]; out is bf16 [M, 3D]; amax_out[r*H+h]
+ *                 receives the max |bf16 value| of region r (q,k,v), head h.
+ *  SWIGLU         W holds 2F rows in the KL_ROWS_SWIGLU_INTERLEAVE order (each
+ *                 128-row group: 64 gate rows then the matching 64 up rows);
+ *                 out[m, f] = bf16(silu(g) * u), silu(g) = g / (1 + e^-g),
+ *                 out is [M, F], F = N/2; amax_out[0] = max |out|.
+ *  GATED_RESIDUAL out = bf16(residual + gate[n] * C).
+ * Shapes: K % 64 == 0; N % 128 == 0 (N % 384 for QKV, % 256 for SWIGLU); any M >= 1.
+ * ([P1] How it works: "kernels fuse ... SwiGLU activations and rotary position
+ * embeddings"; the gated residual is the adaLN reading above.)
+ */
+kl_status kl_gemm_nvfp4_fused(const kl_nvfp4_tensor* A, const kl_nvfp4_tensor* W,
+                              int64_t M, int64_t N, int64_t K, const kl_epilogue* epi,
+                              void* stream);
+
+/*
+ * kl_rope_table -- fp32 (cos, sin) table [T, 64, 2] for the joint sequence
+ * [text (n_text); noisy image (grid_h x grid_w, row-major); n_ref references
+ * on grids of the same size].  Reading (RoPE theta 10000 on head dim 128,
+ * interleaved pairs): text token i turns pair j by i*theta^(-2j/128); an
+ * image-family token at (f, r, c) -- f = 0 for the noisy image, f = k for
+ * reference k -- turns pairs [0,16) by f*theta^(-2u/32), [16,40) by
+ * r*theta^(-2u/48), [40,64) by c*theta^(-2u/48) (u = pair index inside the
+ * section).  Angles and cos/sin are evaluated in fp64 on the device and
+ * rounded to fp32.  [P4] The VAE and Tokenization gives the 64x64 grid.
+ */
+typedef struct kl_token_layout {
+  int64_t n_text;
+  int64_t grid_h;
+  int64_t grid_w;
+  int64_t n_ref;
+} kl_token_layout;
+int64_t kl_layout_tokens(const kl_token_layout* layout);
+kl_status kl_rope_table(const kl_token_layout* layout, float theta, float* cs_out, void* stream);
+
+/*
+ * kl_cast_fp8_per_head -- x bf16 [T, ncols] (row stride ld elements), cols in
+ * heads of 128: s[h] = amax[h]/448 (1 if amax[h]==0) and
+ * out[t, c] = e4m3_rne_satfinite(x[t,c] * (448/amax[h])), out row stride ld.
+ * amax: fp32 [ncols/128] (e.g. the QKV epilogue's amax_out); scales_out: fp32
+ * [ncols/128] decode scales.  ([P1] How it works: FP8 query/key/value.)
+ */
+kl_status kl_cast_fp8_per_head(const void* x_bf16, int64_t T, int64_t ncols, int64_t ld,
+                               const float* amax, void* out_e4m3, float* scales_out,
+                               void* stream);
+
+/*
+ * kl_joint_attention_fp8 -- O = softmax(Q K^T / sqrt(128)) V per head over all
+ * T tokens (joint, unmasked: [P4] Two-Stage Processing; [P2] Summary).
+ * q, k, v: [T, H, 128] with row stride ld elements (e.g. the three column
+ * blocks of one [T, 3*H*128] buffer with ld = 3*H*128).
+ *  KL_ATTN_FP8  : E4M3 inputs with per-head decode scales scale_q/k/v [H];
+ *                 S = (q8.k8) * sq*sk; probabilities are normalised by the
+ *                 running row max, multiplied by 256, rounded to E4M3 and fed
+ *                 to the P.V MMA; the row sum uses the unrounded values;
+ *                 O = (P8.V8) * sv / (256 * l).
+ *  KL_ATTN_BF16 : bf16 inputs, scales ignored (may be NULL); P rounded to bf16.
+ * out: bf16 [T, H*128] (row stride H*128).  amax_out (nullable): max|out| is
+ * max-accumulated into it (caller zero-fills).  head_dim must be 128;
+ * ld % 64 == 0.
+ */
+#define KL_ATTN_FP8 0
+#define KL_ATTN_BF16 1
+kl_status kl_joint_attention_fp8(const void* q, const void* k, const void* v, int64_t ld,
+                                 const float* scale_q, const float* scale_k, const float* scale_v,
+                                 int64_t T, int64_t H, int64_t head_dim, int precision,
+                                 void* out_bf16, float* amax_out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * The joint block
+ * ---------------------------------------------------------------------- */
+typedef struct kl_block_weights {
+  kl_nvfp4_tensor wqkv; /* [3D, D]  rows: q (D), k (D), v (D)                      */
+  kl_nvfp4_tensor wo;   /* [D, D]                                                  */
+  kl_nvfp4_tensor w1;   /* [2F, D] in KL_ROWS_SWIGLU_INTERLEAVE order (gate, up)   */
+  kl_nvfp4_tensor w2;   /* [D, F]                                                  */
+} kl_block_weights;
+
+typedef struct kl_block_io {
+  const void* x;        /* bf16 [T, D] input residual stream                       */
+  const void* mod[6];   /* bf16 [D] each: shift1, scale1, gate1, shift2, scale2, gate2 */
+  const float* rope_cs; /* fp32 [T, 64, 2] from kl_rope_table                       */
+  int64_t T, D, H, F;
+  int attn_precision;   /* KL_ATTN_FP8 or KL_ATTN_BF16                             */
+  void* out;            /* bf16 [T, D] block output (must not alias x)             */
+  void* const* stage_events; /* optional (NULL): KL_BLOCK_STAGES+1 cudaEvent_t handles
+                                owned by the caller; events[i] is recorded on the
+                                stream before stage i, events[KL_BLOCK_STAGES] after
+                                the last stage (per-kernel device timing)            */
+} kl_block_io;
+
+/* Stages of kl_joint_block_forward, in launch order (stage_events index). */
+#define KL_STAGE_LN1 0         /* LayerNorm1 + modulate + NVFP4 (2 kernels)       */
+#define KL_STAGE_QKV 1         /* QKV GEMM + RoPE epilogue                        */
+#define KL_STAGE_FP8_CAST 2    /* per-head E4M3 cast (FP8 attention only)         */
+#define KL_STAGE_ATTN 3        /* joint attention                                 */
+#define KL_STAGE_QUANT_O 4     /* NVFP4 of O                                      */
+#define KL_STAGE_OUT 5         /* output-projection GEMM + gated residual         */
+#define KL_STAGE_LN2 6         /* LayerNorm2 + modulate + NVFP4 (2 kernels)       */
+#define KL_STAGE_MLP_UP 7      /* MLP-up GEMM + SwiGLU epilogue                   */
+#define KL_STAGE_QUANT_H 8     /* NVFP4 of h                                      */
+#define KL_STAGE_MLP_DOWN 9    /* MLP-down GEMM + gated residual                  */
+#define KL_BLOCK_STAGES 10
+
+size_t kl_block_workspace_size(int64_t T, int64_t D, int64_t H, int64_t F, int attn_precision);
+
+/*
+ * kl_joint_block_forward -- one joint transformer block ([P2] Summary; [P4]
+ * Two-Stage Processing), plain reading of the wiring:
+ *   m1  = bf16(LN(x)*(1+scale1)+shift1)            -> NVFP4 (dynamic gs)
+ *   qkv = m1 . Wqkv^T, RoPE on q,k, bf16            (QKV_ROPE epilogue)
+ *   [FP8: per-head E4M3 cast of q, k, v]
+ *   O   = joint attention over all T tokens, bf16   -> NVFP4
+ *   x1  = bf16(x + gate1 * (O . Wo^T))              (GATED_RESIDUAL)
+ *   m2  = bf16(LN(x1)*(1+scale2)+shift2)            -> NVFP4
+ *   h   = bf16(silu(g)*u), [g u] = m2 . W1^T        (SWIGLU) -> NVFP4
+ *   out = bf16(x1 + gate2 * (h . W2^T))             (GATED_RESIDUAL)
+ * D = 128*H (H <= 64); F % 128 == 0; T >= 1.
+ * workspace: >= kl_block_workspace_size(...), 256-byte aligned.
+ */
+kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* io,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KLEIN_H */

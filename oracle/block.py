@@ -184,34 +184,61 @@ def attention(q, k, v, rows=None, chunk=1024):
 
 
 def fp8_head_scales(x):
-    """Per-head E4M3 scale s_h = amax_h / 448 (fp32) of x [T, H, d]; 1 if amax is 0."""
+    """Per-head E4M3 decode scale s_h = amax_h / 448 and encode multiplier
+    448 / amax_h (both fp32; 1 and 1 when amax_h is 0) of x [T, H, d]."""
     amax = np.max(np.abs(np.asarray(x, np.float32)), axis=(0, 2)).astype(np.float32)
-    s = (amax / np.float32(448.0)).astype(np.float32)
-    return np.where(amax > 0, s, np.float32(1.0)).astype(np.float32)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0))
+    s = np.where(nz, (safe / np.float32(448.0)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+    inv = np.where(nz, (np.float32(448.0) / safe).astype(np.float32), np.float32(1.0)).astype(np.float32)
+    return s, inv
 
 
-def attention_fp8_emulated(q, k, v, p_scale=256.0):
-    """Diagnostic emulation of FP8 attention (not a contract).
+def fp8_encode_heads(x):
+    """E4M3 values (decoded, unscaled) of x * (448 / amax_h), and the decode
+    scales s_h: x is approximated by e4m3 * s_h."""
+    s, inv = fp8_head_scales(x)
+    y = (np.asarray(x, np.float32) * inv[None, :, None]).astype(np.float32)
+    return e4m3_round(y), s
 
-    Q/K/V are rounded to E4M3 after dividing by their per-head scale; the
-    row-normalised-by-max probabilities exp(s - max) are rounded to E4M3 after
-    multiplying by ``p_scale`` and divided by it again; the row sum uses the
-    unrounded probabilities.
+
+def attention_fp8_emulated(q, k, v, tile=128, p_scale=256.0, rows=None):
+    """FP8 joint attention as a flash-style kernel computes it (a reading; the
+    pages name FP8 Q/K/V attention but not its arithmetic).
+
+    Q, K and V are rounded to E4M3 after scaling each head by 448 / amax.
+    Keys are visited in tiles of ``tile``; per query row a running maximum m
+    of the scaled log2 scores t = (q8 . k8) * sq * sk * log2(e) / sqrt(d) is
+    kept, the tile's probabilities p = 2^(t - m) are multiplied by
+    ``p_scale``, rounded to E4M3 and multiplied with v8, and both the output
+    and the row sum l (of the unrounded p) are rescaled by 2^(m_old - m_new)
+    whenever m grows.  O = acc * s_v / (p_scale * l).  Everything else fp64.
+    ``rows`` optionally restricts the query rows (scales still use all rows).
     """
-    out_heads = []
-    sq, sk, sv = fp8_head_scales(q), fp8_head_scales(k), fp8_head_scales(v)
-    q8 = e4m3_round(np.asarray(q, np.float32) / sq[None, :, None]) * sq[None, :, None]
-    k8 = e4m3_round(np.asarray(k, np.float32) / sk[None, :, None]) * sk[None, :, None]
-    v8 = e4m3_round(np.asarray(v, np.float32) / sv[None, :, None]) * sv[None, :, None]
+    q8, sq = fp8_encode_heads(q)
+    k8, sk = fp8_encode_heads(k)
+    v8, sv = fp8_encode_heads(v)
     T, H, d = q8.shape
+    if rows is not None:
+        q8 = q8[np.asarray(rows)]
+    R = q8.shape[0]
+    out = np.empty((R, H, d), dtype=np.float64)
     for h in range(H):
-        s = (q8[:, h, :] @ k8[:, h, :].T) / np.sqrt(d)
-        s -= s.max(axis=1, keepdims=True)
-        p = np.exp(s)
-        l = p.sum(axis=1, keepdims=True)
-        p8 = e4m3_round(p * p_scale) / p_scale
-        out_heads.append((p8 @ v8[:, h, :]) / l)
-    return np.stack(out_heads, axis=1)
+        c = np.log2(np.e) / np.sqrt(d) * float(sq[h]) * float(sk[h])
+        m = np.full(R, -np.inf)
+        l = np.zeros(R)
+        acc = np.zeros((R, d))
+        for j0 in range(0, T, tile):
+            t = (q8[:, h, :] @ k8[j0:j0 + tile, h, :].T) * c
+            m_new = np.maximum(m, t.max(axis=1))
+            alpha = np.exp2(m - m_new)
+            p = np.exp2(t - m_new[:, None])
+            p8 = e4m3_round(p * p_scale)
+            l = l * alpha + p.sum(axis=1)
+            acc = acc * alpha[:, None] + p8 @ v8[j0:j0 + tile, h, :]
+            m = m_new
+        out[:, h, :] = acc * float(sv[h]) / (p_scale * l[:, None])
+    return out
 
 
 # ---------------------------------------------------------------------------

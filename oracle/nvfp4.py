@@ -70,6 +70,17 @@ def quantize(x, gs=None):
         raise ValueError("quantize: expected [R, C] with C a multiple of 16")
     R, C = x.shape
     gs = global_scale(x) if gs is None else np.float32(gs)
+    # rows are independent once gs is fixed: encode in row chunks (memory only)
+    step = max(1, (1 << 20) // max(C, 1))
+    if R > step:
+        parts = [_quantize_rows(x[r:r + step], gs) for r in range(0, R, step)]
+        return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts]), np.float32(gs))
+    return _quantize_rows(x, gs)
+
+
+def _quantize_rows(x, gs):
+    """Steps 3-7 for the rows of x with the global scale gs already fixed."""
+    R, C = x.shape
     with np.errstate(over="ignore", divide="ignore", under="ignore", invalid="ignore"):
         d6 = np.float32(E2M1_MAX * gs)
         inv = np.float32(np.float32(1.0) / d6)

@@ -1,0 +1,109 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function
+that include/klein.h declares, and its host-side validation / size logic
+answers without touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import diffusion_transformer_image_nvfp4_b200 as kl
+from diffusion_transformer_image_nvfp4_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "klein.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(kl_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kl.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "kl_joint_block_forward" in names and "kl_quantize_nvfp4" in names
+    assert "kl_gemm_nvfp4_fused" in names and "kl_joint_attention_fp8" in names
+    for n in names:
+        assert hasattr(L, n), n
+    # and the binding declares a signature for each
+    assert set(names) <= set(kl._SIGS)
+
+
+def test_status_strings_and_version(L):
+    assert L.kl_status_string(0) == b"KL_OK"
+    assert L.kl_status_string(6) == b"KL_ERR_DEVICE_TIMEOUT"
+    assert L.kl_status_string(99) == b"KL_ERR_UNKNOWN"
+    assert L.kl_version() >= 100
+
+
+def test_scale_and_workspace_sizes(L):
+    assert L.kl_nvfp4_scales_bytes(320, 512, kl.KL_SCALE_LINEAR) == 320 * 32
+    assert L.kl_nvfp4_scales_bytes(320, 512, kl.KL_SCALE_MMA) == 384 * 32      # padded to 128 rows
+    assert L.kl_quantize_workspace_size() >= 4
+    ws = L.kl_block_workspace_size(8704, 3072, 24, 9216, 0)
+    T, D, F = 8704, 3072, 9216
+    assert ws >= T * 3 * D * 2 + T * 3 * D + 2 * T * D * 2 + T * F * 2 + T * F // 2
+    assert L.kl_block_workspace_size(8704, 3072, 24, 9216, 1) < ws            # no FP8 copy in BF16 mode
+    assert L.kl_block_workspace_size(0, 3072, 24, 9216, 0) == 0
+
+
+def test_layout_tokens(L):
+    lay = kl._TokenLayout(512, 64, 64, 1)
+    assert L.kl_layout_tokens(ctypes.byref(lay)) == 8704
+    lay = kl._TokenLayout(512, 64, 64, 4)
+    assert L.kl_layout_tokens(ctypes.byref(lay)) == 20992
+    lay = kl._TokenLayout(-1, 64, 64, 0)
+    assert L.kl_layout_tokens(ctypes.byref(lay)) == -1
+
+
+def test_validation_rejects_bad_arguments_before_any_device_work(L):
+    # null pointers
+    assert L.kl_quantize_nvfp4(None, 4, 64, None, None, None, 0, None, 0, None) == 1
+    fake = 1 << 20   # never dereferenced: every call below fails validation first
+    # unsupported shapes
+    assert L.kl_quantize_nvfp4(fake, 4, 24, fake, fake, fake, 0, fake, 256, None) == 2
+    assert L.kl_quantize_nvfp4(fake, 4, 80, fake, fake, fake, kl.KL_SCALE_MMA, fake, 256, None) == 2
+    assert L.kl_quantize_nvfp4(fake, 100, 64, fake, fake, fake, kl.KL_ROWS_SWIGLU_INTERLEAVE, fake, 256, None) == 2
+    # misaligned input
+    assert L.kl_quantize_nvfp4(fake + 2, 4, 64, fake, fake, fake, 0, fake, 256, None) == 3
+    # missing workspace when gs is derived
+    assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, 0, None, 0, None) == 4
+    # bad flag bits
+    assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, 64, fake, 256, None) == 1
+    # GEMM shape and epilogue checks
+    t = kl._NVFP4Tensor(fake, fake, fake)
+    epi = kl._Epilogue(0, 0, fake, None, None, None, None)
+    assert L.kl_gemm_nvfp4_fused(ctypes.byref(t), ctypes.byref(t), 128, 100, 64, ctypes.byref(epi), None) == 2
+    assert L.kl_gemm_nvfp4_fused(ctypes.byref(t), ctypes.byref(t), 128, 128, 96, ctypes.byref(epi), None) == 2
+    epi_q = kl._Epilogue(1, 0, fake, None, None, None, None)
+    assert L.kl_gemm_nvfp4_fused(ctypes.byref(t), ctypes.byref(t), 128, 384, 64, ctypes.byref(epi_q), None) == 1
+    epi_bad = kl._Epilogue(9, 0, fake, None, None, None, None)
+    assert L.kl_gemm_nvfp4_fused(ctypes.byref(t), ctypes.byref(t), 128, 128, 64, ctypes.byref(epi_bad), None) == 1
+    # attention
+    assert L.kl_joint_attention_fp8(fake, fake, fake, 3072, None, None, None, 100, 24, 128, 0, fake, None, None) == 1
+    assert L.kl_joint_attention_fp8(fake, fake, fake, 3072, fake, fake, fake, 100, 24, 64, 0, fake, None, None) == 2
+    assert L.kl_joint_attention_fp8(fake, fake, fake, 3072, fake, fake, fake, 100, 24, 128, 7, fake, None, None) == 1
+    # block: D must be 128 * H
+    io = kl._BlockIO(fake, (ctypes.c_void_p * 6)(*([fake] * 6)), fake, 100, 3000, 24, 9216, 0, fake + 4096)
+    w = kl._BlockWeights(t, t, t, t)
+    assert L.kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), fake, 1 << 40, None) == 2
+    io.D = 3072
+    io.out = fake
+    assert L.kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), fake, 1 << 40, None) == 1  # out aliases x
+    io.out = fake + 4096
+    assert L.kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), fake, 16, None) == 4     # workspace
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(kl, "_LIB", None)
+    monkeypatch.setattr(kl, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        kl.lib()

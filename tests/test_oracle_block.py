@@ -297,3 +297,32 @@ def test_block_runs_on_tiny_workload():
     assert out.shape == (wl.n_tokens, wl.hidden) and np.isfinite(out).all()
     # branch deltas are non-trivial
     assert np.abs(inter["x1"] - inp["x"]).max() > 0
+
+
+def test_fp8_emulation_uniform_scores_give_mean_of_quantised_values():
+    # q = 0 makes every score 0, every p exactly 1 (p * 256 = 256 is an E4M3
+    # value), so O is the plain mean of the E4M3-decoded v, over any tiling
+    rng = np.random.default_rng(12)
+    T, H = 300, 2
+    q = np.zeros((T, H, 128))
+    k = rng.standard_normal((T, H, 128))
+    v = rng.standard_normal((T, H, 128)).astype(np.float32)
+    o = block.attention_fp8_emulated(q, k, v)
+    v8, sv = block.fp8_encode_heads(v)
+    want = (v8 * sv[None, :, None]).mean(axis=0)
+    np.testing.assert_allclose(o, np.broadcast_to(want, o.shape), rtol=1e-12, atol=1e-15)
+    o2 = block.attention_fp8_emulated(q, k, v, tile=64)
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-15)
+
+
+def test_fp8_emulation_close_to_exact_and_rows_subset():
+    rng = np.random.default_rng(13)
+    q, k, v = (rng.standard_normal((260, 2, 128)) for _ in range(3))
+    exact, _ = block.attention(q, k, v)
+    emu = block.attention_fp8_emulated(q, k, v)
+    err = np.linalg.norm(emu - exact) / np.linalg.norm(exact)
+    assert 0.0 < err < 0.08
+    rows = np.array([0, 5, 259])
+    np.testing.assert_allclose(block.attention_fp8_emulated(q, k, v, rows=rows), emu[rows], rtol=1e-13)
+    s, inv = block.fp8_head_scales(v)
+    np.testing.assert_allclose(s * inv, 1.0, rtol=1e-6)
