@@ -79,7 +79,9 @@ def test_bf16_output_and_single_block_operand():
     got = to_np(kl.gemm_nvfp4_fused(A, W))
     ref = codecs.bf16_round(_ref(a, w))
     assert np.all(got[:129] == 0)
-    np.testing.assert_allclose(got, ref, rtol=2 ** -7, atol=0)
+    # row 129 sums 16 products per output: a cancelling sum can leave fp32
+    # accumulation noise where the fp64 sum is ~0, hence the absolute term
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2 ** -7 + 1e-5 * _bound(a, w))
 
 
 def test_gated_residual_epilogue():
