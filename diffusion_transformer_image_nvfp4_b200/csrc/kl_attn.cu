@@ -8,20 +8,22 @@
 // Image Klein inference on NVIDIA Blackwell GPUs", How it works ("Quantized
 // attention uses FP8 precision for query, key, and value").
 //
-// One CTA = one 128-query tile of one head (192 threads, one CTA per SM):
-//  * warp 0 lane 0 -- TMA: the Q tile once, then K and V tiles of 128 keys
-//    into a 4-stage (FP8) / 2-stage (BF16) ring, 128-byte swizzle;
-//  * warp 1 lane 0 -- MMA: S_j = Q K_j^T into one of two TMEM score buffers,
-//    then O_j = P_j V_j into one of two TMEM output buffers (V read MN-major
-//    straight from its row-major tile); the score MMA of tile j+1 is issued
-//    before the P.V MMA of tile j so the tensor core works while the softmax
-//    warps exponentiate;
-//  * warps 2-5 -- softmax (thread = query row): row max over S_j (pass 1),
-//    p = 2^(s*c - m) (pass 2), P written to smem in the MMA's K-major swizzled
-//    layout (FP8: p*256 rounded to E4M3), running row sum l from the unrounded
-//    p; O_j is folded into a register accumulator O = O*2^(m_old-m_new) + O_j.
-//    Output O / l (times s_v/256 in FP8 mode) as bf16, plus a tensor amax.
-// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
+// One CTA = QT query tiles of 128 rows of one head (FP8: QT = 2, BF16: 1):
+//  * warp 0 lane 0 -- TMA: the Q tiles once, then K and V tiles of 128 keys
+//    into a ring (FP8: 3 stages, BF16: 2), 128-byte swizzle;
+//  * warp 1 lane 0 -- MMA: per key tile j and query tile t, S_t = Q_t K_j^T
+//    into TMEM; then O_t += P_t V_{j-1} (V read MN-major straight from its
+//    row-major tile) for the previous key tile, so the tensor core computes
+//    the next scores while the softmax warps exponentiate;
+//  * 4 softmax warps per query tile (thread = query row): one pass over the
+//    scores in registers; the running maximum m is only moved (and O, l
+//    rescaled in place -- O in TMEM after the previous P.V has landed) when a
+//    tile's maximum exceeds m by more than TAU (log2 units), so
+//    p = 2^(s*c - m) <= 2^TAU; p * P_SCALE is rounded to E4M3 (BF16: bf16)
+//    and written to a double-buffered smem P tile in the MMA's K-major
+//    swizzled layout; l sums the unrounded p.
+//    Finally O = O_tmem / l (FP8: times s_v / P_SCALE), bf16, and a tensor amax.
+// TMEM per query tile: S [128 cols] + O [128 cols].
 #include "kl_common.cuh"
 #include "kl_internal.h"
 
@@ -31,7 +33,7 @@ struct AttnParams {
   int64_t T;
   int H;
   int n_kv;
-  float c_log2;        // BF16: log2(e)/sqrt(128); FP8: times sq*sk (per head, applied in kernel)
+  float c_log2;  // log2(e)/sqrt(128); FP8: times sq*sk (per head, in the kernel)
   const float* sq;
   const float* sk;
   const float* sv;
@@ -42,14 +44,19 @@ struct AttnParams {
 template <bool FP8>
 struct AttnCfg {
   static constexpr int ELEM = FP8 ? 1 : 2;
-  static constexpr int TILE = 128 * 128 * ELEM;  // Q, K, V or P tile bytes
-  static constexpr int NS = FP8 ? 4 : 2;
-  static constexpr int KSTEPS = FP8 ? 4 : 8;     // MMA K = 32 (e4m3) or 16 (bf16)
+  static constexpr int QT = FP8 ? 2 : 1;           // query tiles per CTA
+  static constexpr int TILE = 128 * 128 * ELEM;    // Q, K, V or P tile bytes
+  static constexpr int NS = FP8 ? 3 : 2;           // K/V ring stages
+  static constexpr int KSTEPS = FP8 ? 4 : 8;       // MMA K = 32 (e4m3) or 16 (bf16)
+  static constexpr float TAU = FP8 ? 4.0f : 8.0f;  // lazy-rescale threshold, log2 units
+  static constexpr float P_SCALE = FP8 ? 16.0f : 1.0f;  // p * P_SCALE <= 2^(TAU+4) <= 448
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = TILE;
+  static constexpr int KV_OFF = QT * TILE;
   static constexpr int P_OFF = KV_OFF + NS * 2 * TILE;
-  static constexpr int BAR_OFF = P_OFF + 2 * TILE;
-  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+  static constexpr int BAR_OFF = P_OFF + QT * 2 * TILE;
+  static constexpr int THREADS = 64 + QT * 128;
+  static constexpr uint32_t TMEM_COLS = QT * 256;
+  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
   static_assert(SMEM_BYTES <= 232448, "smem budget");
 };
 
@@ -73,28 +80,29 @@ __device__ __forceinline__ void tma_tile(uint8_t* dst, const CUtensorMap* map, i
 }
 
 template <bool FP8>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const AttnParams p) {
   using C = AttnCfg<FP8>;
+  constexpr int QT = C::QT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + C::NS;
-  uint64_t* s_full = kv_empty + C::NS;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_full = p_empty + 2;
-  uint64_t* o_empty = o_full + 2;
-  uint64_t* drain = o_empty + 2;
+  uint64_t* q_full = bars;                    // 1
+  uint64_t* kv_full = q_full + 1;             // NS
+  uint64_t* kv_empty = kv_full + C::NS;       // NS
+  uint64_t* s_full = kv_empty + C::NS;        // QT
+  uint64_t* s_empty = s_full + QT;            // QT
+  uint64_t* p_full = s_empty + QT;            // QT x 2
+  uint64_t* p_empty = p_full + 2 * QT;        // QT x 2
+  uint64_t* o_done = p_empty + 2 * QT;        // QT: one phase per P.V
+  uint64_t* o_last = o_done + QT;             // QT: the last P.V only
+  uint64_t* drain = o_last + QT;              // 1
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y;
+  const int qblk = blockIdx.x, h = blockIdx.y;
   const int n = p.n_kv;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -102,20 +110,22 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4);
-      mbar_init(&p_full[b], 4);
-      mbar_init(&p_empty[b], 1);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_empty[b], 4);
+    for (int t = 0; t < QT; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_empty[t], 4);
+      mbar_init(&o_done[t], 1);
+      mbar_init(&o_last[t], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&p_full[2 * t + b], 4);
+        mbar_init(&p_empty[2 * t + b], 1);
+      }
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -132,8 +142,8 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tmap(&tq);
       prefetch_tmap(&tk);
       prefetch_tmap(&tv);
-      mbar_arrive_expect_tx(q_full, C::TILE);
-      tma_tile<FP8>(q_smem, &tq, h * 128, qt * 128, q_full);
+      mbar_arrive_expect_tx(q_full, QT * C::TILE);
+      for (int t = 0; t < QT; ++t) tma_tile<FP8>(q_smem + t * C::TILE, &tq, h * 128, (qblk * QT + t) * 128, q_full);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
@@ -163,48 +173,57 @@ __global__ void __launch_bounds__(192, 1)
       // ------------------------------------------------------------ MMA
       const uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
       const uint32_t id_pv = FP8 ? idesc_e4m3(128, 128, 1) : idesc_bf16(128, 128, 1);
-      const uint32_t q_addr = smem_u32(q_smem);
       bool ok = mbar_wait(q_full, 0, abort_flag);
       for (int j = 0; ok && j <= n; ++j) {
         if (j < n) {
-          const int s = j % C::NS, b = j & 1;
-          if (!mbar_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag) ||
-              !mbar_wait(&s_empty[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) {
+          const int s = j % C::NS;
+          if (!mbar_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t k_addr = smem_u32(kv_smem + s * 2 * C::TILE);
+          for (int t = 0; t < QT && ok; ++t) {
+            if (!mbar_wait(&s_empty[t], ((uint32_t)j & 1u) ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(q_smem + t * C::TILE);
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint64_t ad = kmajor_desc<FP8>(q_addr, kk), bd = kmajor_desc<FP8>(k_addr, kk);
-            if (FP8)
-              mma_f8(tmem + b * 128, ad, bd, id_qk, kk > 0);
-            else
-              mma_f16(tmem + b * 128, ad, bd, id_qk, kk > 0);
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t ad = kmajor_desc<FP8>(q_addr, kk), bd = kmajor_desc<FP8>(k_addr, kk);
+              if (FP8)
+                mma_f8(tmem + t * 256, ad, bd, id_qk, kk > 0);
+              else
+                mma_f16(tmem + t * 256, ad, bd, id_qk, kk > 0);
+            }
+            tc_commit(&s_full[t]);
           }
-          tc_commit(&s_full[b]);
+          if (!ok) break;
         }
         if (j >= 1) {
           const int jj = j - 1, s = jj % C::NS, b = jj & 1;
-          const uint32_t ph = (uint32_t)(jj >> 1) & 1u;
-          if (!mbar_wait(&p_full[b], ph, abort_flag) || !mbar_wait(&o_empty[b], ph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t p_addr = smem_u32(p_smem + b * C::TILE);
           const uint32_t v_addr = smem_u32(kv_smem + s * 2 * C::TILE + C::TILE);
+          for (int t = 0; t < QT && ok; ++t) {
+            if (!mbar_wait(&p_full[2 * t + b], (uint32_t)(jj >> 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t p_addr = smem_u32(p_smem + (2 * t + b) * C::TILE);
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint64_t ad = kmajor_desc<FP8>(p_addr, kk), bd = vdesc<FP8>(v_addr, kk);
-            if (FP8)
-              mma_f8(tmem + 256 + b * 128, ad, bd, id_pv, kk > 0);
-            else
-              mma_f16(tmem + 256 + b * 128, ad, bd, id_pv, kk > 0);
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t ad = kmajor_desc<FP8>(p_addr, kk), bd = vdesc<FP8>(v_addr, kk);
+              if (FP8)
+                mma_f8(tmem + t * 256 + 128, ad, bd, id_pv, (jj | kk) != 0);
+              else
+                mma_f16(tmem + t * 256 + 128, ad, bd, id_pv, (jj | kk) != 0);
+            }
+            tc_commit(&o_done[t]);
+            tc_commit(&p_empty[2 * t + b]);
+            if (jj == n - 1) tc_commit(&o_last[t]);
           }
-          tc_commit(&o_full[b]);
-          tc_commit(&p_empty[b]);
+          if (!ok) break;
           tc_commit(&kv_empty[s]);
         }
       }
@@ -214,128 +233,132 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // query row inside the tile
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const int sw = warp - 2;              // softmax warp 0 .. 4*QT-1
+    const int t = sw >> 2;                // query tile of this warp
+    const int quad = warp & 3;            // TMEM lane group this warp may access
+    const int r = quad * 32 + lane;       // query row inside the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(t * 256);
+    const uint32_t s_tmem = lane_base, o_tmem = lane_base + 128;
     float c = p.c_log2;
     if (FP8) c *= __ldg(p.sq + h) * __ldg(p.sk + h);
-    float o[128];
-#pragma unroll
-    for (int i = 0; i < 128; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
-
-    auto combine = [&](int i, float a) -> bool {
-      const int b = i & 1;
-      if (!mbar_wait(&o_full[b], (uint32_t)(i >> 1) & 1u, abort_flag)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(lane_base + 256 + b * 128 + cc * 32, v);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) o[cc * 32 + t] = fmaf(o[cc * 32 + t], a, v[t]);
+    for (int j = 0; j < n; ++j) {
+      if (!warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag)) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      float sc[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_tmem + cc * 32, *reinterpret_cast<float(*)[32]>(sc + cc * 32));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[b]);
-      return true;
-    };
-
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-      if (!mbar_wait(&s_full[b], ph, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      if (lane == 0) mbar_arrive(&s_empty[t]);
       const int64_t rem = p.T - (int64_t)j * 128;
-      const int valid = rem < 128 ? (int)rem : 128;
-      float mx = -INFINITY;
+      if (rem < 128) {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(lane_base + b * 128 + cc * 32, v);
-#pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (cc * 32 + t < valid) mx = fmaxf(mx, v[t]);
+        for (int i = 0; i < 128; ++i)
+          if (i >= rem) sc[i] = -INFINITY;
       }
-      const float m_new = fmaxf(m, mx * c);
-      const float alpha = ex2_approx(m - m_new);
-      if (!mbar_wait(&p_empty[b], ph ^ 1u, abort_flag)) {
+      float mx = sc[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sc[i]);
+      mx *= c;
+      // this P buffer was last read by P.V of key tile j-2: once it is free,
+      // every P.V up to j-2 has landed
+      const int b = j & 1;
+      if (!warp_wait(&p_empty[2 * t + b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-      uint8_t* prow = p_smem + b * C::TILE + r * 128;
+      const bool move = mx > m + C::TAU;
+      if (__any_sync(0xffffffffu, move)) {
+        // move the reference maximum of the rows that need it and rescale
+        // their O (in TMEM, after P.V of tile j-1 has landed) and l by
+        // 2^(m_old - m_new).  TMEM loads/stores are warp-wide, so the whole
+        // warp takes this path; rows that do not move use a factor of 1.
+        const float alpha = move ? ex2_approx(m - mx) : 1.0f;
+        if (j > 0) {
+          if (!warp_wait(&o_done[t], (uint32_t)(j - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float o[32];
+            tmem_ld32(o_tmem + cc * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(o_tmem + cc * 32, o);
+          }
+          tc_fence_before();
+        }
+        l *= alpha;
+        if (move) m = mx;
+      }
+      uint8_t* prow = p_smem + (2 * t + b) * C::TILE + r * 128;
       float rowsum = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(lane_base + b * 128 + cc * 32, v);
+      for (int i = 0; i < 128; ++i) {
+        sc[i] = ex2_approx(fmaf(sc[i], c, -m));
+        rowsum += sc[i];
+      }
+      if (FP8) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float pv = (cc * 32 + t < valid) ? ex2_approx(fmaf(v[t], c, -m_new)) : 0.f;
-          rowsum += pv;
-          v[t] = pv;
-        }
-        if (FP8) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t w[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float* x = v + hh * 16 + q * 4;
-              w[q] = f32x2_to_e4m3x2(x[0] * 256.f, x[1] * 256.f) | (f32x2_to_e4m3x2(x[2] * 256.f, x[3] * 256.f) << 16);
-            }
-            const int chunk = cc * 2 + hh;
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else {
+        for (int chunk = 0; chunk < 8; ++chunk) {
+          uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float* x = v + q * 8;
-            const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                                       pack_bf16x2(x[6], x[7]));
-            const int chunk = (cc & 1) * 4 + q;
-            *reinterpret_cast<uint4*>(prow + (cc >> 1) * 16384 + ((chunk ^ (r & 7)) << 4)) = w;
+            const float* x = sc + chunk * 16 + q * 4;
+            w[q] = f32x2_to_e4m3x2(x[0] * C::P_SCALE, x[1] * C::P_SCALE) |
+                   (f32x2_to_e4m3x2(x[2] * C::P_SCALE, x[3] * C::P_SCALE) << 16);
           }
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else {
+#pragma unroll
+        for (int chunk = 0; chunk < 16; ++chunk) {
+          const float* x = sc + chunk * 8;
+          const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                     pack_bf16x2(x[6], x[7]));
+          *reinterpret_cast<uint4*>(prow + (chunk >> 3) * 16384 + (((chunk & 7) ^ (r & 7)) << 4)) = w;
         }
       }
-      tc_fence_before();
+      l += rowsum;
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_empty[b]);
-        mbar_arrive(&p_full[b]);
-      }
-      l = fmaf(l, alpha, rowsum);
-      if (j >= 1 && !combine(j - 1, alpha_prev)) {
-        ok = false;
-        break;
-      }
-      alpha_prev = alpha;
-      m = m_new;
+      if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
     }
-    if (ok) ok = combine(n - 1, alpha_prev);
-    // epilogue: O / l, bf16, tensor amax
-    const int64_t row = (int64_t)qt * 128 + r;
+    // epilogue: O / l (FP8: times s_v / P_SCALE), bf16, tensor amax
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) ok = warp_wait(&o_last[t], 0, abort_flag);
+    const int64_t row = ((int64_t)qblk * QT + t) * 128 + r;
     const bool valid_row = ok && row < p.T;
     float scale = 1.0f / l;
-    if (FP8) scale *= __ldg(p.sv + h) * (1.0f / 256.0f);
+    if (FP8) scale *= __ldg(p.sv + h) * (1.0f / C::P_SCALE);
     float amax = 0.f;
-    uint4* dst = reinterpret_cast<uint4*>(p.out + row * (int64_t)p.H * 128 + h * 128);
+    if (ok) {
+      tc_fence_after();
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * (int64_t)p.H * 128 + h * 128);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        tmem_ld32(o_tmem + cc * 32, o);
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      float x[8];
+        for (int q = 0; q < 4; ++q) {
+          float x[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        x[t] = bf16_bits_to_f32(f32_to_bf16_bits(o[q * 8 + t] * scale));
-        amax = fmaxf(amax, fabsf(x[t]));
+          for (int i = 0; i < 8; ++i) {
+            x[i] = bf16_bits_to_f32(f32_to_bf16_bits(o[q * 8 + i] * scale));
+            amax = fmaxf(amax, fabsf(x[i]));
+          }
+          if (valid_row)
+            dst[cc * 4 + q] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                         pack_bf16x2(x[6], x[7]));
+        }
       }
-      if (valid_row)
-        dst[q] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                            pack_bf16x2(x[6], x[7]));
     }
     if (p.amax) {
       amax = warp_max(valid_row ? amax : 0.f);
@@ -347,7 +370,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -374,8 +397,9 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
   p.amax = a.amax;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)p.n_kv, (unsigned)a.H);
-  attn_kernel<FP8><<<grid, 192, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  const int qblocks = (int)((a.T + 128 * C::QT - 1) / (128 * C::QT));
+  dim3 grid((unsigned)qblocks, (unsigned)a.H);
+  attn_kernel<FP8><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,7 @@
 // fuse SwiGLU activations and rotary position embeddings.  The page names
 // those kernels (PrimsTS) but gives no design; this one is written for B200:
 //
-//  * persistent grid (one 192-thread CTA per SM), 128 x BN output tiles,
+//  * persistent grid (one 320-thread CTA per SM), 128 x BN output tiles,
 //    BN = 256 (one TMEM accumulator) or 128 (two, so the epilogue of tile i
 //    overlaps the main loop of tile i+1);
 //  * warp 0 lane 0: TMA producer.  A [128 x 256] and W [BN x 256] FP4 tiles
@@ -19,8 +19,10 @@
 //  * warp 1 lane 0: MMA issuer.  Per 64-wide K step: tcgen05.cp of the A and
 //    W scale atoms into TMEM, then one 128 x BN x 64 block-scaled MMA into the
 //    TMEM accumulator; tcgen05.commit releases smem stages / publishes tiles;
-//  * warps 2-5: epilogue.  tcgen05.ld 32 columns at a time (thread = row),
-//    scale by gA*gW, apply the fused epilogue, store bf16/fp32.
+//  * warps 2-9: epilogue (thread = row, two warps per 32-lane TMEM group,
+//    one per half of the tile's columns).  The whole accumulator is drained
+//    to registers with tcgen05.ld and released before the math, so scaling by
+//    gA*gW, the fused epilogue and the stores overlap the next tile's MMAs.
 // Smem ring: 4 (BN 256) or 6 (BN 128) stages of ~54 / 36 KB.
 #include "kl_common.cuh"
 #include "kl_internal.h"
@@ -93,7 +95,7 @@ __device__ __forceinline__ float round_bf16x32(float (&v)[32]) {
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < C::ACC; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -233,69 +235,91 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // 8 warps: warp w reads TMEM lanes 32*(w%4).. (its rows) and one half of
+    // the tile's columns.  Each tile is first drained into registers and the
+    // accumulator released at once, so the math and stores below overlap the
+    // next tile's MMAs.
+    constexpr int HALF = BN / 2;        // accumulator columns per thread
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_in_tile = quad * 32 + lane;
     const float alpha = __fmul_rn(__ldg(p.gsa), __ldg(p.gsw));
     const int64_t D = p.N / 3;           // QKV only
     const int H = (int)(D >> 7);
     int acc = 0;
     uint32_t acc_phase = 0;
+    float v[HALF];
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      if (!warp_wait(&tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int64_t row = (int64_t)mb * 128 + row_in_tile;
       const bool valid = row < p.M;
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
       const int64_t n0 = (int64_t)nb * BN;
       if (p.epi == KL_EPI_SWIGLU) {
-        float amax = 0.f;
-        const int64_t F = p.N >> 1;
-#pragma unroll 1
-        for (int g = 0; g < BN / 128; ++g) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < 64; c0 += 32) {
-            float vg[32], vu[32];
-            tmem_ld32(tbase + g * 128 + c0, vg);
-            tmem_ld32(tbase + g * 128 + 64 + c0, vu);
+        // this thread's outputs o in [half*BN/4, (half+1)*BN/4): gate column
+        // (o/64)*128 + o%64 of the tile, up column = gate column + 64
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float gg = vg[i] * alpha, uu = vu[i] * alpha;
-              vg[i] = gg / (1.0f + expf(-gg)) * uu;
-            }
-            amax = fmaxf(amax, round_bf16x32(vg));
-            if (valid)
-              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + g * 64 + c0, vg);
+        for (int c = 0; c < BN / 4; c += 32) {
+          const int o0 = half * (BN / 4) + c;
+          const int gcol = (o0 >> 6) * 128 + (o0 & 63);
+          tmem_ld32(tbase + gcol, *reinterpret_cast<float(*)[32]>(v + c));
+          tmem_ld32(tbase + gcol + 64, *reinterpret_cast<float(*)[32]>(v + BN / 4 + c));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < HALF; c += 32) tmem_ld32(tbase + half * HALF + c, *reinterpret_cast<float(*)[32]>(v + c));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == C::ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+#pragma unroll
+      for (int i = 0; i < HALF; ++i) v[i] *= alpha;
+
+      if (p.epi == KL_EPI_SWIGLU) {
+        const int64_t F = p.N >> 1;
+        float amax = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN / 4; c += 32) {
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gg = v[c + i], uu = v[BN / 4 + c + i];
+            h[i] = gg / (1.0f + expf(-gg)) * uu;
           }
+          amax = fmaxf(amax, round_bf16x32(h));
+          if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + half * (BN / 4) + c, h);
         }
         amax = warp_max(valid ? amax : 0.f);
         if (lane == 0) atomic_max_nonneg(p.amax, amax);
       } else {
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          float v[32];
-          tmem_ld32(tbase + c0, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          const int64_t n = n0 + c0;
+        for (int c = 0; c < HALF; c += 32) {
+          float* w = v + c;
+          const int64_t n = n0 + half * HALF + c;
           if (p.epi == KL_EPI_NONE) {
             if (valid) {
               if (p.out_f32) {
                 float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.N + n);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                for (int q = 0; q < 8; ++q) d[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
               } else {
-                store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+                store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
               }
             }
           } else if (p.epi == KL_EPI_GATED_RESIDUAL) {
-            float gt[32], rs[32];
-            load_bf16x32(p.gate + n, gt);
             if (valid) {
+              float gt[32], rs[32];
+              load_bf16x32(p.gate + n, gt);
               load_bf16x32(p.residual + row * p.N + n, rs);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __fmaf_rn(gt[i], v[i], rs[i]);
-              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+              for (int i = 0; i < 32; ++i) w[i] = __fmaf_rn(gt[i], w[i], rs[i]);
+              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
             }
           } else {  // KL_EPI_QKV_ROPE
             const int region = (int)(n / D);
@@ -307,26 +331,19 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
                 const float4 t = __ldg(cs + q);  // (c, s) of two consecutive pairs
-                const float a0 = v[4 * q], b0 = v[4 * q + 1], a1 = v[4 * q + 2], b1 = v[4 * q + 3];
-                v[4 * q] = a0 * t.x - b0 * t.y;
-                v[4 * q + 1] = a0 * t.y + b0 * t.x;
-                v[4 * q + 2] = a1 * t.z - b1 * t.w;
-                v[4 * q + 3] = a1 * t.w + b1 * t.z;
+                const float a0 = w[4 * q], b0 = w[4 * q + 1], a1 = w[4 * q + 2], b1 = w[4 * q + 3];
+                w[4 * q] = a0 * t.x - b0 * t.y;
+                w[4 * q + 1] = a0 * t.y + b0 * t.x;
+                w[4 * q + 2] = a1 * t.z - b1 * t.w;
+                w[4 * q + 3] = a1 * t.w + b1 * t.z;
               }
             }
-            float amax = round_bf16x32(v);
-            if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, v);
+            float amax = round_bf16x32(*reinterpret_cast<float(*)[32]>(w));
+            if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
             amax = warp_max(valid ? amax : 0.f);
             if (lane == 0) atomic_max_nonneg(p.amax + region * H + head, amax);
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (++acc == C::ACC) {
-        acc = 0;
-        acc_phase ^= 1u;
       }
     }
   }
@@ -372,7 +389,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  gemm_nvfp4_kernel<BN><<<grid, 192, C::SMEM_BYTES, s>>>(ta, tb, p);
+  gemm_nvfp4_kernel<BN><<<grid, 320, C::SMEM_BYTES, s>>>(ta, tb, p);
   return cudaGetLastError();
 }
 

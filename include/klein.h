@@ -220,11 +220,14 @@ kl_status kl_cast_fp8_per_head(const void* x_bf16, int64_t T, int64_t ncols, int
  * q, k, v: [T, H, 128] with row stride ld elements (e.g. the three column
  * blocks of one [T, 3*H*128] buffer with ld = 3*H*128).
  *  KL_ATTN_FP8  : E4M3 inputs with per-head decode scales scale_q/k/v [H];
- *                 S = (q8.k8) * sq*sk; probabilities are normalised by the
- *                 running row max, multiplied by 256, rounded to E4M3 and fed
- *                 to the P.V MMA; the row sum uses the unrounded values;
- *                 O = (P8.V8) * sv / (256 * l).
- *  KL_ATTN_BF16 : bf16 inputs, scales ignored (may be NULL); P rounded to bf16.
+ *                 S = (q8.k8) * sq*sk.  Keys are taken in tiles of 128; per
+ *                 query row a reference maximum m (log2 units) moves only when
+ *                 a tile's maximum exceeds it by more than 4, and then the
+ *                 partial output and row sum are rescaled, so p = 2^(s - m) <=
+ *                 16; p * 16 is rounded to E4M3 and fed to the P.V MMA; the row
+ *                 sum l uses the unrounded p; O = (P8.V8) * sv / (16 * l).
+ *  KL_ATTN_BF16 : bf16 inputs, scales ignored (may be NULL); the same scheme
+ *                 with threshold 8 and P rounded to bf16 (no extra scale).
  * out: bf16 [T, H*128] (row stride H*128).  amax_out (nullable): max|out| is
  * max-accumulated into it (caller zero-fills).  head_dim must be 128;
  * ld % 64 == 0.

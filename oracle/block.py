@@ -202,17 +202,18 @@ def fp8_encode_heads(x):
     return e4m3_round(y), s
 
 
-def attention_fp8_emulated(q, k, v, tile=128, p_scale=256.0, rows=None):
+def attention_fp8_emulated(q, k, v, tile=128, p_scale=16.0, tau=4.0, rows=None):
     """FP8 joint attention as a flash-style kernel computes it (a reading; the
     pages name FP8 Q/K/V attention but not its arithmetic).
 
     Q, K and V are rounded to E4M3 after scaling each head by 448 / amax.
-    Keys are visited in tiles of ``tile``; per query row a running maximum m
-    of the scaled log2 scores t = (q8 . k8) * sq * sk * log2(e) / sqrt(d) is
-    kept, the tile's probabilities p = 2^(t - m) are multiplied by
-    ``p_scale``, rounded to E4M3 and multiplied with v8, and both the output
-    and the row sum l (of the unrounded p) are rescaled by 2^(m_old - m_new)
-    whenever m grows.  O = acc * s_v / (p_scale * l).  Everything else fp64.
+    Keys are visited in tiles of ``tile``.  Per query row a reference maximum
+    m of the scaled log2 scores t = (q8 . k8) * sq * sk * log2(e) / sqrt(d) is
+    kept; it is only moved -- and the output accumulator and row sum l are
+    rescaled by 2^(m_old - m_new) -- when a tile's maximum exceeds m by more
+    than ``tau``, so every p = 2^(t - m) <= 2^tau.  p * ``p_scale`` is rounded
+    to E4M3 and multiplied with v8; l sums the unrounded p.
+    O = acc * s_v / (p_scale * l).  Everything else fp64.
     ``rows`` optionally restricts the query rows (scales still use all rows).
     """
     q8, sq = fp8_encode_heads(q)
@@ -230,13 +231,16 @@ def attention_fp8_emulated(q, k, v, tile=128, p_scale=256.0, rows=None):
         acc = np.zeros((R, d))
         for j0 in range(0, T, tile):
             t = (q8[:, h, :] @ k8[j0:j0 + tile, h, :].T) * c
-            m_new = np.maximum(m, t.max(axis=1))
-            alpha = np.exp2(m - m_new)
-            p = np.exp2(t - m_new[:, None])
+            mx = t.max(axis=1)
+            move = mx > m + tau
+            alpha = np.where(move, np.exp2(np.where(move, m - mx, 0.0)), 1.0)
+            acc *= alpha[:, None]
+            l *= alpha
+            m = np.where(move, mx, m)
+            p = np.exp2(t - m[:, None])
             p8 = e4m3_round(p * p_scale)
-            l = l * alpha + p.sum(axis=1)
-            acc = acc * alpha[:, None] + p8 @ v8[j0:j0 + tile, h, :]
-            m = m_new
+            l += p.sum(axis=1)
+            acc += p8 @ v8[j0:j0 + tile, h, :]
         out[:, h, :] = acc * float(sv[h]) / (p_scale * l[:, None])
     return out
 
