@@ -79,6 +79,7 @@ _SIGS = {
     "kl_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _I, _VP, _SZ, _VP], _I),
     "kl_ln_workspace_size": ([_I64], _SZ),
     "kl_ln_modulate_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
+    "kl_ln_modulate_quantize_nvfp4_static": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "kl_gemm_nvfp4_fused": ([ctypes.POINTER(_NVFP4Tensor), ctypes.POINTER(_NVFP4Tensor), _I64, _I64, _I64,
                              ctypes.POINTER(_Epilogue), _VP], _I),
     "kl_layout_tokens": ([ctypes.POINTER(_TokenLayout)], _I64),
@@ -190,6 +191,24 @@ def ln_modulate_quantize_nvfp4(x, shift, scale, export_m=False):
     _check(L.kl_ln_modulate_quantize_nvfp4(x.data_ptr(), R, C, shift.data_ptr(), scale.data_ptr(), codes.data_ptr(),
                                            scales.data_ptr(), gs.data_ptr(), _ptr(m), ws.data_ptr(), ws.numel(),
                                            _stream()), "kl_ln_modulate_quantize_nvfp4")
+    q = NVFP4(codes, scales, gs, R, C, "mma")
+    return (q, m) if export_m else q
+
+
+def ln_modulate_quantize_nvfp4_static(x, shift, scale, export_m=False):
+    """kl_ln_modulate_quantize_nvfp4_static: as ln_modulate_quantize_nvfp4, but
+    the library's scratch comes from its own fixed device array (no workspace)."""
+    for t, n in ((x, "x"), (shift, "shift"), (scale, "scale")):
+        _need(t, torch.bfloat16, n)
+    R, C = x.shape
+    L = lib()
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, KL_SCALE_MMA), dtype=torch.uint8, device=x.device)
+    gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    m = torch.empty_like(x) if export_m else None
+    _check(L.kl_ln_modulate_quantize_nvfp4_static(x.data_ptr(), R, C, shift.data_ptr(), scale.data_ptr(),
+                                                  codes.data_ptr(), scales.data_ptr(), gs.data_ptr(), _ptr(m),
+                                                  _stream()), "kl_ln_modulate_quantize_nvfp4_static")
     q = NVFP4(codes, scales, gs, R, C, "mma")
     return (q, m) if export_m else q
 

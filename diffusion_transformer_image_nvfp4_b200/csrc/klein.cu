@@ -4,3 +4,4 @@
 #include "kl_gemm.cu"
 #include "kl_attn.cu"
 #include "kl_api.cu"
+#include "kl_noalloc.cu"

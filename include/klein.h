@@ -132,6 +132,34 @@ kl_status kl_ln_modulate_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_
                                         void* m_out_bf16, void* workspace, size_t ws_bytes,
                                         void* stream);
 
+/*
+ * kl_ln_modulate_quantize_nvfp4_static -- the same computation, arguments and
+ * outputs as kl_ln_modulate_quantize_nvfp4, without the workspace.  The pages
+ * have no counterpart: this exists for callers that cannot give the library
+ * any device memory, e.g. a host that plans and owns the whole device pool up
+ * front and forbids allocations after start-up, or a plugin interface that
+ * passes only input and output buffers.  The call allocates nothing (no
+ * cudaMalloc / cudaFree, no allocating library routine).
+ *  - Scratch (one amax word + 8 bytes of LayerNorm statistics per row) lives
+ *    in a fixed device array compiled into the library:
+ *    256 + 8 * KL_STATIC_SCRATCH_MAX_ROWS bytes (= 262,400), held on every GPU
+ *    that loads the library until the process exits.
+ *  - rows > KL_STATIC_SCRATCH_MAX_ROWS is rejected with KL_ERR_WORKSPACE
+ *    (kl_last_cuda_error() names the limit) before anything is enqueued.
+ *  - The first call on a device looks up that array's device address
+ *    (cudaGetSymbolAddress) with the device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    each call zeroes the amax word on its stream before use.  Calls that
+ *    overlap on the same GPU (e.g. issued on two streams) race on it:
+ *    serialise them.  Each device has its own copy of the array.
+ */
+#define KL_STATIC_SCRATCH_MAX_ROWS 32768
+kl_status kl_ln_modulate_quantize_nvfp4_static(const void* x_bf16, int64_t rows, int64_t cols,
+                                               const void* shift_bf16, const void* scale_bf16,
+                                               void* codes, void* scales, float* global_scale,
+                                               void* m_out_bf16, void* stream);
+
 /* An NVFP4 GEMM operand: codes [R, K/2], scales in KL_SCALE_MMA layout,
  * global decode scale (device fp32). */
 typedef struct kl_nvfp4_tensor {

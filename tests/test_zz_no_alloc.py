@@ -1,0 +1,61 @@
+"""kl_ln_modulate_quantize_nvfp4_static -- the allocation-free variant of the
+fused LayerNorm + adaLN + NVFP4 encoder, for callers that cannot give the
+library device memory (a host that owns the whole device pool, a plugin
+interface that passes only inputs and outputs).
+
+It is called here through the C ABI (ctypes, raw device pointers) and must
+give exactly what the workspace entry point kl_ln_modulate_quantize_nvfp4
+gives, on two calls in a row with different inputs (the fixed scratch array
+keeps the previous call's amax and statistics, which must not leak).  This
+file is collected last so a stop-at-first-failure run has already run every
+other test; it passes alone in a fresh process too.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import diffusion_transformer_image_nvfp4_b200 as kl
+from synth import normal_bf16
+
+
+def _static_call(x, shift, scale):
+    L = kl.lib()
+    R, C = x.shape
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, kl.KL_SCALE_MMA), dtype=torch.uint8, device=x.device)
+    gs = torch.empty(1, dtype=torch.float32, device=x.device)
+    m = torch.empty_like(x)
+    st = L.kl_ln_modulate_quantize_nvfp4_static(
+        ctypes.c_void_p(x.data_ptr()), R, C, ctypes.c_void_p(shift.data_ptr()), ctypes.c_void_p(scale.data_ptr()),
+        ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(gs.data_ptr()),
+        ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, L.kl_status_string(st)
+    return codes, scales, gs, m
+
+
+@pytest.mark.gpu
+def test_static_scratch_matches_workspace_entry_point_on_two_calls():
+    cases = [((4608, 3072), 1, 30.0), ((333, 512), 2, 0.05)]   # big amax first, then a small one
+    for (rows, cols), seed, std in cases:
+        x = normal_bf16((rows, cols), seed, std).cuda()
+        shift = normal_bf16((cols,), seed + 10, 0.1).cuda()
+        scale = normal_bf16((cols,), seed + 20, 0.1).cuda()
+        codes, scales, gs, m = _static_call(x, shift, scale)
+        ref, m_ref = kl.ln_modulate_quantize_nvfp4(x, shift, scale, export_m=True)
+        torch.cuda.synchronize()
+        assert gs.cpu().numpy().tobytes() == ref.gs.cpu().numpy().tobytes()
+        np.testing.assert_array_equal(scales.cpu().numpy(), ref.scales.cpu().numpy())
+        np.testing.assert_array_equal(codes.cpu().numpy(), ref.codes.cpu().numpy())
+        np.testing.assert_array_equal(m.view(torch.int16).cpu().numpy(), m_ref.view(torch.int16).cpu().numpy())
+    assert kl.device_status() == "KL_OK"
+
+
+def test_static_scratch_rejects_rows_beyond_its_capacity():
+    L = kl.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the size check comes first
+    st = L.kl_ln_modulate_quantize_nvfp4_static(fake, 32769, 512, fake, fake, fake, fake, fake, None, None)
+    assert L.kl_status_string(st) == b"KL_ERR_WORKSPACE"
+    assert b"32768" in L.kl_last_cuda_error()
