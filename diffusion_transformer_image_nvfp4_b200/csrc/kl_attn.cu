@@ -21,8 +21,8 @@
 //    tile's maximum exceeds m by more than TAU (log2 units), so
 //    p = 2^(s*c - m) <= 2^TAU; p * P_SCALE is rounded to E4M3 (BF16: bf16)
 //    and written to a double-buffered smem P tile in the MMA's K-major
-//    swizzled layout; l sums the unrounded p.
-//    Finally O = O_tmem / l (FP8: times s_v / P_SCALE), bf16, and a tensor amax.
+//    swizzled layout; l sums the unrounded p * P_SCALE.
+//    Finally O = O_tmem / l (FP8: times s_v), bf16, and a tensor amax.
 // TMEM per query tile: S [128 cols] + O [128 cols].
 #include "kl_common.cuh"
 #include "kl_internal.h"
@@ -50,6 +50,7 @@ struct AttnCfg {
   static constexpr int KSTEPS = FP8 ? 4 : 8;       // MMA K = 32 (e4m3) or 16 (bf16)
   static constexpr float TAU = FP8 ? 4.0f : 8.0f;  // lazy-rescale threshold, log2 units
   static constexpr float P_SCALE = FP8 ? 16.0f : 1.0f;  // p * P_SCALE <= 2^(TAU+4) <= 448
+  static constexpr float LOG2_P_SCALE = FP8 ? 4.0f : 0.0f;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = QT * TILE;
   static constexpr int P_OFF = KV_OFF + NS * 2 * TILE;
@@ -261,10 +262,15 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (i >= rem) sc[i] = -INFINITY;
       }
-      float mx = sc[0];
+      // row maximum: 8 independent chains of 3-input max
+      float mk[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sc[i]);
-      mx *= c;
+      for (int k = 0; k < 8; ++k) mk[k] = fmaxf(sc[2 * k], sc[2 * k + 1]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], sc[i + 2 * k], sc[i + 2 * k + 1]);
+      float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7])) * c;
       // this P buffer was last read by P.V of key tile j-2: once it is free,
       // every P.V up to j-2 has landed
       const int b = j & 1;
@@ -299,12 +305,24 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
         if (move) m = mx;
       }
       uint8_t* prow = p_smem + (2 * t + b) * C::TILE + r * 128;
-      float rowsum = 0.f;
+      // p * P_SCALE = 2^(s*c - (m - log2 P_SCALE)); packed fp32x2 FMAs, and
+      // the row sum (of the scaled p) in 4 independent packed chains
+      const uint64_t c2 = pack_f32x2(c, c);
+      const float mb = -(m - C::LOG2_P_SCALE);
+      const uint64_t mb2 = pack_f32x2(mb, mb);
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        sc[i] = ex2_approx(fmaf(sc[i], c, -m));
-        rowsum += sc[i];
+      for (int i = 0; i < 128; i += 2) {
+        float lo, hi;
+        unpack_f32x2(fma_f32x2(pack_f32x2(sc[i], sc[i + 1]), c2, mb2), lo, hi);
+        sc[i] = ex2_approx(lo);
+        sc[i + 1] = ex2_approx(hi);
+        acc2[(i >> 1) & 3] = add_f32x2(acc2[(i >> 1) & 3], pack_f32x2(sc[i], sc[i + 1]));
       }
+      float a0, a1, b0, b1;
+      unpack_f32x2(add_f32x2(acc2[0], acc2[1]), a0, a1);
+      unpack_f32x2(add_f32x2(acc2[2], acc2[3]), b0, b1);
+      const float rowsum = (a0 + a1) + (b0 + b1);
       if (FP8) {
 #pragma unroll
         for (int chunk = 0; chunk < 8; ++chunk) {
@@ -312,8 +330,7 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float* x = sc + chunk * 16 + q * 4;
-            w[q] = f32x2_to_e4m3x2(x[0] * C::P_SCALE, x[1] * C::P_SCALE) |
-                   (f32x2_to_e4m3x2(x[2] * C::P_SCALE, x[3] * C::P_SCALE) << 16);
+            w[q] = f32x2_to_e4m3x2(x[0], x[1]) | (f32x2_to_e4m3x2(x[2], x[3]) << 16);
           }
           *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -331,13 +348,13 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
     }
-    // epilogue: O / l (FP8: times s_v / P_SCALE), bf16, tensor amax
+    // epilogue: O / l (FP8: times s_v), bf16, tensor amax
     ok = __all_sync(0xffffffffu, ok);
     if (ok) ok = warp_wait(&o_last[t], 0, abort_flag);
     const int64_t row = ((int64_t)qblk * QT + t) * 128 + r;
     const bool valid_row = ok && row < p.T;
-    float scale = 1.0f / l;
-    if (FP8) scale *= __ldg(p.sv + h) * (1.0f / C::P_SCALE);
+    float scale = 1.0f / l;  // l sums p * P_SCALE, so this also undoes P_SCALE
+    if (FP8) scale *= __ldg(p.sv + h);
     float amax = 0.f;
     if (ok) {
       tc_fence_after();

@@ -9,16 +9,19 @@
 // fuse SwiGLU activations and rotary position embeddings.  The page names
 // those kernels (PrimsTS) but gives no design; this one is written for B200:
 //
-//  * persistent grid (one 320-thread CTA per SM), 128 x BN output tiles,
+//  * persistent grid (one 352-thread CTA per SM), 128 x BN output tiles,
 //    BN = 256 (one TMEM accumulator) or 128 (two, so the epilogue of tile i
 //    overlaps the main loop of tile i+1);
 //  * warp 0 lane 0: TMA producer.  A [128 x 256] and W [BN x 256] FP4 tiles
 //    (128 bytes per row, 128-byte swizzle) by cp.async.bulk.tensor; the block
 //    scales for those tiles, already stored in the MMA scale layout, by
 //    cp.async.bulk (contiguous 512-byte atoms);
-//  * warp 1 lane 0: MMA issuer.  Per 64-wide K step: tcgen05.cp of the A and
-//    W scale atoms into TMEM, then one 128 x BN x 64 block-scaled MMA into the
-//    TMEM accumulator; tcgen05.commit releases smem stages / publishes tiles;
+//  * warp 10 lane 0: scale copier.  Per 64-wide K step, tcgen05.cp of the A
+//    and W scale atoms into the stage's own TMEM scale buffer, ahead of the
+//    MMA issuer (tcgen05.commit -> sf_ready);
+//  * warp 1 lane 0: MMA issuer.  One 128 x BN x 64 block-scaled MMA per K
+//    step into the TMEM accumulator; tcgen05.commit releases smem stages and
+//    publishes finished tiles;
 //  * warps 2-9: epilogue (thread = row, two warps per 32-lane TMEM group,
 //    one per half of the tile's columns).  The whole accumulator is drained
 //    to registers with tcgen05.ld and released before the math, so scaling by
@@ -55,11 +58,14 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int ACC = BN == 256 ? 1 : 2;
-  static constexpr uint32_t SFA_COL = ACC * BN;
-  static constexpr uint32_t SFB_COL = SFA_COL + 16;
+  // block scales: one TMEM buffer per smem stage (SFA 16 columns, SFB
+  // 4*BN/32), so the scale copy of a K tile never waits for the MMAs of an
+  // earlier K tile to finish reading the previous scales
+  static constexpr uint32_t SF_COLS = 16 + 4 * (BN / 32);
+  static constexpr uint32_t SF_BASE = ACC * BN;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-  static_assert(SFB_COL + 4 * (BN / 32) <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "smem budget");
 };
 
@@ -95,7 +101,7 @@ __device__ __forceinline__ float round_bf16x32(float (&v)[32]) {
 }
 
 template <int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const GemmParams p) {
   using C = GemmCfg<BN>;
@@ -105,8 +111,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + C::ACC;
-  uint64_t* drain = tempty + C::ACC;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = tempty + C::ACC;   // STAGES: scales of the stage are in TMEM
+  uint64_t* drain = sf_ready + C::STAGES;  // 2: MMA issuer, scale copier
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,12 +121,14 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     for (int a = 0; a < C::ACC; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 8);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -192,28 +201,22 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          // the operand tiles have landed and the scale-copy warp has moved
+          // this stage's block scales into the stage's TMEM scale buffer
+          if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_ready[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint8_t* sa = smem + stage * C::STAGE_BYTES;
           const uint8_t* sb = sa + C::A_BYTES;
-          const uint8_t* ssfa = sb + C::B_BYTES;
-          const uint8_t* ssfb = ssfa + C::SFA_BYTES;
           const int nk = min(4, p.kbn - kt * 4);
-          for (int kk = 0; kk < nk; ++kk) {
-            tmem_cp_32x128b_x4(tmem + C::SFA_COL + kk * 4, smem_desc(smem_u32(ssfa + kk * 512), 0, 128, kLayoutNone));
-#pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              tmem_cp_32x128b_x4(tmem + C::SFB_COL + kk * (BN / 32) + j * 4,
-                                 smem_desc(smem_u32(ssfb + j * 2048 + kk * 512), 0, 128, kLayoutNone));
-          }
+          const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 16;
           for (int kk = 0; kk < nk; ++kk) {
             const uint64_t ad = smem_desc(smem_u32(sa + kk * 32), 16, 1024, kLayoutSw128);
             const uint64_t bd = smem_desc(smem_u32(sb + kk * 32), 16, 1024, kLayoutSw128);
-            mma_nvf4(d_tmem, ad, bd, idesc, tmem + C::SFA_COL + kk * 4, tmem + C::SFB_COL + kk * (BN / 32),
-                     (kt | kk) != 0 ? 1u : 0u);
+            mma_nvf4(d_tmem, ad, bd, idesc, sfa_t + kk * 4, sfb_t + kk * (BN / 32), (kt | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -228,10 +231,51 @@ __global__ void __launch_bounds__(320, 1)
           acc_phase ^= 1u;
         }
       }
-      // every MMA / copy issued by this thread has completed before TMEM is freed
-      tc_commit(drain);
+      // every MMA issued by this thread has completed before TMEM is freed
+      tc_commit(&drain[0]);
       volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort);
+      mbar_wait(&drain[0], 0, &no_abort);
+    }
+  } else if (warp == 10) {
+    // -------------------------------------------------------- scale copier
+    // Moves each stage's block scales from smem into that stage's TMEM scale
+    // buffer as soon as the stage lands, ahead of the MMA issuer, so the MMA
+    // thread issues only MMAs.  A stage (and its scale buffer) is refilled
+    // only after the MMAs that read it have completed (empty -> producer ->
+    // full), so the copies never overwrite scales still in use.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* ssfa = smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+          const uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          const int nk = min(4, p.kbn - kt * 4);
+          const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 16;
+          for (int kk = 0; kk < nk; ++kk) {
+            tmem_cp_32x128b_x4(sfa_t + kk * 4, smem_desc(smem_u32(ssfa + kk * 512), 0, 128, kLayoutNone));
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tmem_cp_32x128b_x4(sfb_t + kk * (BN / 32) + j * 4,
+                                 smem_desc(smem_u32(ssfb + j * 2048 + kk * 512), 0, 128, kLayoutNone));
+          }
+          tc_commit(&sf_ready[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      tc_commit(&drain[1]);
+      volatile int no_abort = 0;
+      mbar_wait(&drain[1], 0, &no_abort);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -257,7 +301,11 @@ __global__ void __launch_bounds__(320, 1)
       const bool valid = row < p.M;
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
       const int64_t n0 = (int64_t)nb * BN;
-      if (p.epi == KL_EPI_SWIGLU) {
+      if constexpr (BN == 256) {
+        // columns [128*half, 128*half + 128): for SwiGLU that is exactly one
+        // 64-gate + 64-up row group, already in the order used below
+        tmem_ld128(tbase + half * 128, v);
+      } else if (p.epi == KL_EPI_SWIGLU) {
         // this thread's outputs o in [half*BN/4, (half+1)*BN/4): gate column
         // (o/64)*128 + o%64 of the tile, up column = gate column + 64
 #pragma unroll
@@ -289,8 +337,11 @@ __global__ void __launch_bounds__(320, 1)
           float h[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
+            // silu(g) * u with the fast exp / divide intrinsics (relative
+            // error ~1e-6, far below the bf16 rounding of h); the argument
+            // is clamped so the denominator stays finite
             const float gg = v[c + i], uu = v[BN / 4 + c + i];
-            h[i] = gg / (1.0f + expf(-gg)) * uu;
+            h[i] = __fdividef(gg, 1.0f + __expf(fminf(-gg, 80.0f))) * uu;
           }
           amax = fmaxf(amax, round_bf16x32(h));
           if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + half * (BN / 4) + c, h);
@@ -389,7 +440,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  gemm_nvfp4_kernel<BN><<<grid, 320, C::SMEM_BYTES, s>>>(ta, tb, p);
+  gemm_nvfp4_kernel<BN><<<grid, 352, C::SMEM_BYTES, s>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
