@@ -64,15 +64,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
-                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -297,7 +298,8 @@ kl_status kl_joint_attention_fp8(const void* q, const void* k, const void* v, in
 
 // ------------------------------------------------------------ block driver
 // Workspace layout (each piece 256-byte aligned):
-//   words  : amax[0..3] (m1, O, m2, h), gs[4..7], qkv amax [3H], fp8 scales [3H]
+//   words  : amax[0..3] (O at 1, h at 3), gs[4..7], qkv amax [3H], fp8 scales [3H],
+//            LN1 and LN2 amax words [2 + 2]
 //   stats  : float2 [T]                       LayerNorm mean / rstd
 //   acodes : uint8 [T, D/2], ascales [Tp, D/16]   NVFP4 A operand (m1, then O, then m2)
 //   qkv    : bf16 [T, 3D]
@@ -322,7 +324,7 @@ static BlockWs block_ws_layout(uint8_t* base, int64_t T, int64_t D, int64_t H, i
     off += up256(bytes);
     return p;
   };
-  w.words = reinterpret_cast<float*>(take((8 + 6 * (size_t)H) * sizeof(float)));
+  w.words = reinterpret_cast<float*>(take((12 + 6 * (size_t)H) * sizeof(float)));
   w.stats = reinterpret_cast<float2*>(take((size_t)T * sizeof(float2)));
   w.acodes = take((size_t)T * D / 2);
   w.ascales = take((size_t)Tp * D / 16);
@@ -363,11 +365,13 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   BlockWs ws = block_ws_layout(reinterpret_cast<uint8_t*>(workspace), T, D, H, F, io->attn_precision);
-  float* amax = ws.words;          // [0] m1, [1] O, [2] m2, [3] h
+  float* amax = ws.words;          // [1] O, [3] h (LN amaxes live in ln1 / ln2)
   float* gs = ws.words + 4;        // [0] m1, [1] O, [2] m2, [3] h
   float* amax_qkv = ws.words + 8;  // [3H]
   float* sc8 = amax_qkv + 3 * H;   // [3H]
-  cudaError_t e = cudaMemsetAsync(ws.words, 0, (8 + 6 * H) * sizeof(float), s);
+  float* ln1 = sc8 + 3 * H;        // LN1 amax
+  float* ln2 = ln1 + 2;            // LN2 amax
+  cudaError_t e = cudaMemsetAsync(ws.words, 0, (12 + 6 * H) * sizeof(float), s);
 #define KL_TRY(x)                      \
   do {                                 \
     if (e == cudaSuccess) e = (x);     \
@@ -379,7 +383,7 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   mark(0);
   // 1. m1 = bf16(LN(x)(1+scale1)+shift1) -> NVFP4
   KL_TRY(launch_ln_modulate_quantize(io->x, T, D, io->mod[0], io->mod[1], ws.acodes, ws.ascales, &gs[0], nullptr,
-                                     ws.stats, &amax[0], s));
+                                     ws.stats, ln1, s));
   mark(1);
   // 2. qkv = m1 Wqkv^T with RoPE on q, k and per-head amax
   GemmArgs g{};
@@ -445,7 +449,7 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   mark(6);
   // 7. m2 = bf16(LN(x1)(1+scale2)+shift2) -> NVFP4
   KL_TRY(launch_ln_modulate_quantize(ws.x1, T, D, io->mod[3], io->mod[4], ws.acodes, ws.ascales, &gs[2], nullptr,
-                                     ws.stats, &amax[2], s));
+                                     ws.stats, ln2, s));
   mark(7);
   // 8. h = bf16(silu(g) u), [g u] = m2 W1^T, + amax
   g = GemmArgs{};

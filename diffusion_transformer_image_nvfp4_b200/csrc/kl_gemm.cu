@@ -48,25 +48,32 @@ struct GemmParams {
   int num_m, num_tiles, num_kt, kbn;  // kbn = K / 64
 };
 
-template <int BN>
+// BN: output tile width (256 or 128).  KS: 64-wide K steps per smem stage
+// (4 -> 128-byte operand rows, 128-byte swizzle; 2 -> 64-byte rows, 64-byte
+// swizzle and twice the stages for the same bytes in flight).
+template <int BN, int KS = 4>
 struct GemmCfg {
   static constexpr int BM = 128;
-  static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN * 128;
-  static constexpr int SFA_BYTES = 2048;
-  static constexpr int SFB_BYTES = (BN / 128) * 2048;
+  static constexpr int ROWB = KS * 32;               // operand bytes per row per stage
+  static constexpr int A_BYTES = BM * ROWB;
+  static constexpr int B_BYTES = BN * ROWB;
+  static constexpr int SFA_BYTES = KS * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * KS * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = (220 * 1024) / STAGE_BYTES;
   static constexpr int ACC = BN == 256 ? 1 : 2;
-  // block scales: one TMEM buffer per smem stage (SFA 16 columns, SFB
-  // 4*BN/32), so the scale copy of a K tile never waits for the MMAs of an
-  // earlier K tile to finish reading the previous scales
-  static constexpr uint32_t SF_COLS = 16 + 4 * (BN / 32);
+  static constexpr uint32_t LAYOUT = KS == 4 ? 2u : 4u;   // smem descriptor swizzle: 128 B or 64 B
+  static constexpr uint32_t SBO = 8 * ROWB;               // bytes between 8-row groups
+  // block scales: one TMEM buffer per smem stage (SFA 4*KS columns, SFB
+  // KS*4*BN/128), so the scale copy of a K tile never waits for the MMAs of
+  // an earlier K tile to finish reading the previous scales
+  static constexpr uint32_t SF_COLS = 4 * KS + KS * 4 * (BN / 128);
   static constexpr uint32_t SF_BASE = ACC * BN;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
   static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "smem budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 };
 
 __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32]) {
@@ -100,11 +107,11 @@ __device__ __forceinline__ float round_bf16x32(float (&v)[32]) {
   return m;
 }
 
-template <int BN>
+template <int BN, int KS>
 __global__ void __launch_bounds__(352, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, KS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -163,16 +170,16 @@ __global__ void __launch_bounds__(352, 1)
           uint8_t* sb = sa + C::A_BYTES;
           uint8_t* ssfa = sb + C::B_BYTES;
           uint8_t* ssfb = ssfa + C::SFA_BYTES;
-          const int nk = min(4, p.kbn - kt * 4);
+          const int nk = min(KS, p.kbn - kt * KS);
           const uint32_t sf_bytes = (uint32_t)nk * 512u;
           mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
-          tma_load_2d(sa, &tmap_a, kt * 128, mb * 128, &full[stage]);
-          tma_load_2d(sb, &tmap_b, kt * 128, nb * BN, &full[stage]);
-          bulk_load(ssfa, p.sfa + ((int64_t)mb * p.kbn + kt * 4) * 512, sf_bytes, &full[stage]);
+          tma_load_2d(sa, &tmap_a, kt * C::ROWB, mb * 128, &full[stage]);
+          tma_load_2d(sb, &tmap_b, kt * C::ROWB, nb * BN, &full[stage]);
+          bulk_load(ssfa, p.sfa + ((int64_t)mb * p.kbn + kt * KS) * 512, sf_bytes, &full[stage]);
 #pragma unroll
           for (int j = 0; j < BN / 128; ++j)
-            bulk_load(ssfb + j * 2048, p.sfb + ((int64_t)(nb * (BN / 128) + j) * p.kbn + kt * 4) * 512, sf_bytes,
-                      &full[stage]);
+            bulk_load(ssfb + j * KS * 512, p.sfb + ((int64_t)(nb * (BN / 128) + j) * p.kbn + kt * KS) * 512,
+                      sf_bytes, &full[stage]);
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -210,12 +217,12 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
           const uint8_t* sa = smem + stage * C::STAGE_BYTES;
           const uint8_t* sb = sa + C::A_BYTES;
-          const int nk = min(4, p.kbn - kt * 4);
+          const int nk = min(KS, p.kbn - kt * KS);
           const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
-          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t sfb_t = sfa_t + 4 * KS;
           for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t ad = smem_desc(smem_u32(sa + kk * 32), 16, 1024, kLayoutSw128);
-            const uint64_t bd = smem_desc(smem_u32(sb + kk * 32), 16, 1024, kLayoutSw128);
+            const uint64_t ad = smem_desc(smem_u32(sa + kk * 32), 16, C::SBO, C::LAYOUT);
+            const uint64_t bd = smem_desc(smem_u32(sb + kk * 32), 16, C::SBO, C::LAYOUT);
             mma_nvf4(d_tmem, ad, bd, idesc, sfa_t + kk * 4, sfb_t + kk * (BN / 32), (kt | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
@@ -256,15 +263,15 @@ __global__ void __launch_bounds__(352, 1)
           tc_fence_after();
           const uint8_t* ssfa = smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
           const uint8_t* ssfb = ssfa + C::SFA_BYTES;
-          const int nk = min(4, p.kbn - kt * 4);
+          const int nk = min(KS, p.kbn - kt * KS);
           const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
-          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t sfb_t = sfa_t + 4 * KS;
           for (int kk = 0; kk < nk; ++kk) {
             tmem_cp_32x128b_x4(sfa_t + kk * 4, smem_desc(smem_u32(ssfa + kk * 512), 0, 128, kLayoutNone));
 #pragma unroll
             for (int j = 0; j < BN / 128; ++j)
               tmem_cp_32x128b_x4(sfb_t + kk * (BN / 32) + j * 4,
-                                 smem_desc(smem_u32(ssfb + j * 2048 + kk * 512), 0, 128, kLayoutNone));
+                                 smem_desc(smem_u32(ssfb + j * KS * 512 + kk * 512), 0, 128, kLayoutNone));
           }
           tc_commit(&sf_ready[stage]);
           if (++stage == C::STAGES) {
@@ -407,15 +414,16 @@ __global__ void __launch_bounds__(352, 1)
   }
 }
 
-template <int BN>
+template <int BN, int KS>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, KS>;
   CUtensorMap ta, tb;
+  const int swz = KS == 4 ? 128 : 64;
   if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
-                    (uint64_t)(a.K / 2), 128, 128))
+                    (uint64_t)(a.K / 2), C::ROWB, 128, swz))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                    (uint64_t)(a.K / 2), 128, BN))
+                    (uint64_t)(a.K / 2), C::ROWB, BN, swz))
     return cudaErrorInvalidValue;
   GemmParams p;
   p.M = a.M;
@@ -435,20 +443,24 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
   p.num_m = (int)((a.M + 127) / 128);
   p.num_tiles = p.num_m * (int)(a.N / BN);
   p.kbn = (int)(a.K / 64);
-  p.num_kt = (p.kbn + 3) / 4;
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  p.num_kt = (p.kbn + KS - 1) / KS;
+  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  gemm_nvfp4_kernel<BN><<<grid, 352, C::SMEM_BYTES, s>>>(ta, tb, p);
+  gemm_nvfp4_kernel<BN, KS><<<grid, 352, C::SMEM_BYTES, s>>>(ta, tb, p);
   return cudaGetLastError();
 }
+
+#ifndef KL_GEMM_KSTEPS
+#define KL_GEMM_KSTEPS 4
+#endif
 
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   int bn = a.force_bn;
   if (bn == 0) bn = (a.N % 256 == 0) ? 256 : 128;
   if (bn == 256 && a.N % 256 != 0) return cudaErrorInvalidValue;
-  return bn == 256 ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
+  return bn == 256 ? launch_bn<256, KL_GEMM_KSTEPS>(a, s) : launch_bn<128, KL_GEMM_KSTEPS>(a, s);
 }
 
 }  // namespace kl

@@ -60,7 +60,8 @@ struct AttnArgs {
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
 // tensor maps (kl_api.cu)
+// 2D tensor map, box_inner x box_outer elements, 128-byte (or 64-byte) swizzle
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
-                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes = 128);
 
 }  // namespace kl

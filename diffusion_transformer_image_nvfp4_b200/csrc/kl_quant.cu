@@ -235,6 +235,147 @@ __global__ void __launch_bounds__(256) ln_quant_kernel(const uint16_t* __restric
   }
 }
 
+// ------------------------- LayerNorm + modulate, warp per row, NCH chunks
+// Lane l holds elements [(c*32 + l)*8, +8) of chunk c, c < NCH = cols/256;
+// all NCH 16-byte loads of a row are issued before any arithmetic.
+// Statistics pass: mean, rstd (the same fp32 operation sequence as
+// ln_stats_amax_kernel) and the amax of m, from registers.
+template <int NCH>
+__global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                            const uint16_t* __restrict__ shift,
+                                                            const uint16_t* __restrict__ scale,
+                                                            float2* __restrict__ stats, float* __restrict__ amax) {
+  constexpr int64_t cols = NCH * 256;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+  float lmax = 0.f;
+  if (row < rows) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+    uint4 xv[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) xv[c] = __ldg(xr + c * 32 + lane);
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s += bf16_bits_to_f32(w[j] & 0xFFFFu) + bf16_bits_to_f32(w[j] >> 16);
+    }
+    const float mean = __fdiv_rn(warp_sum(s), (float)cols);
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = bf16_bits_to_f32(w[j] & 0xFFFFu) - mean, b = bf16_bits_to_f32(w[j] >> 16) - mean;
+        ss += a * a + b * b;
+      }
+    }
+    const float rstd = __frsqrt_rn(__fadd_rn(__fdiv_rn(warp_sum(ss), (float)cols), 1e-6f));
+    if (lane == 0) stats[row] = make_float2(mean, rstd);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const uint4 sh = __ldg(reinterpret_cast<const uint4*>(shift) + c * 32 + lane);
+      const uint4 sc = __ldg(reinterpret_cast<const uint4*>(scale) + c * 32 + lane);
+      const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+      const uint32_t a[4] = {sh.x, sh.y, sh.z, sh.w}, b[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t sft = hh ? 16 : 0;
+          const float onep = __fadd_rn(1.0f, bf16_bits_to_f32((b[j] >> sft) & 0xFFFFu));
+          const float mv = ln_mod_value(bf16_bits_to_f32((w[j] >> sft) & 0xFFFFu), mean, rstd, onep,
+                                        bf16_bits_to_f32((a[j] >> sft) & 0xFFFFu));
+          lmax = fmaxf(lmax, fabsf(mv));
+        }
+    }
+  }
+  lmax = warp_max(lmax);
+  if (lane == 0 && row < rows) atomic_max_nonneg(amax, lmax);
+}
+
+// Encode pass: recompute m from x (an L2 re-read) and the stored statistics,
+// 16-element blocks = the 8 elements of lanes 2k and 2k+1 of one chunk.
+template <int NCH>
+__global__ void __launch_bounds__(256) ln_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                            int64_t rows_padded, const uint16_t* __restrict__ shift,
+                                                            const uint16_t* __restrict__ scale,
+                                                            const float2* __restrict__ stats,
+                                                            const float* __restrict__ amax,
+                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                            float* __restrict__ gs_out, uint16_t* __restrict__ m_out) {
+  constexpr int64_t cols = NCH * 256;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+  const GsParams g = gs_from_amax(*amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = g.gs;
+  if (row >= rows_padded) return;
+  if (row >= rows) {  // padding rows of the MMA scale layout
+    for (int64_t kb = lane; kb < (cols >> 4); kb += 32) scales[mma_scale_offset(row, kb, cols)] = 0;
+    return;
+  }
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+  uint4 xv[NCH];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) xv[c] = __ldg(xr + c * 32 + lane);
+  const float2 st = stats[row];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int64_t col = ((int64_t)c * 32 + lane) * 8;
+    const uint4 sh = __ldg(reinterpret_cast<const uint4*>(shift) + c * 32 + lane);
+    const uint4 sc = __ldg(reinterpret_cast<const uint4*>(scale) + c * 32 + lane);
+    const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+    const uint32_t a[4] = {sh.x, sh.y, sh.z, sh.w}, b[4] = {sc.x, sc.y, sc.z, sc.w};
+    float v[8];
+    float a8 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t sft = hh ? 16 : 0;
+        const float onep = __fadd_rn(1.0f, bf16_bits_to_f32((b[j] >> sft) & 0xFFFFu));
+        v[2 * j + hh] = ln_mod_value(bf16_bits_to_f32((w[j] >> sft) & 0xFFFFu), st.x, st.y, onep,
+                                     bf16_bits_to_f32((a[j] >> sft) & 0xFFFFu));
+        a8 = fmaxf(a8, fabsf(v[2 * j + hh]));
+      }
+    if (m_out)
+      *reinterpret_cast<uint4*>(m_out + row * cols + col) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    const float amax_b = fmaxf(a8, __shfl_xor_sync(0xffffffffu, a8, 1));
+    const uint32_t sb = amax_b > 0.f ? f32_to_e4m3(__fmul_rn(amax_b, g.inv)) : 0u;
+    const float S = __fmul_rn(e4m3_to_f32(sb), g.gs);
+    uint32_t code = 0u;
+    if (S != 0.f) {
+      const float rr = __fdiv_rn(1.0f, S);
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], rr);
+      code = f32x8_to_e2m1x8(y);
+    }
+    *reinterpret_cast<uint32_t*>(codes + row * (cols >> 1) + (col >> 1)) = code;
+    if ((lane & 1) == 0) scales[mma_scale_offset(row, col >> 4, cols)] = (uint8_t)sb;
+  }
+}
+
+template <int NCH>
+static cudaError_t launch_ln_rows(const void* x, int64_t rows, const void* shift, const void* scale, void* codes,
+                                  void* scales, float* gs_out, void* m_out, float2* stats, float* amax,
+                                  cudaStream_t s) {
+  const uint16_t* xp = reinterpret_cast<const uint16_t*>(x);
+  const uint16_t* shp = reinterpret_cast<const uint16_t*>(shift);
+  const uint16_t* scp = reinterpret_cast<const uint16_t*>(scale);
+  ln_stats_rows_kernel<NCH><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(xp, rows, shp, scp, stats, amax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t rows_padded = ((rows + 127) / 128) * 128;
+  ln_quant_rows_kernel<NCH><<<(unsigned)((rows_padded + 7) / 8), 256, 0, s>>>(
+      xp, rows, rows_padded, shp, scp, stats, amax, reinterpret_cast<uint8_t*>(codes),
+      reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ FP8 cast
 // 16 elements per thread (inside one 128-wide head).
 __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t ncols,
@@ -315,6 +456,18 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
                                         void* m_out, float2* stats, float* amax, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return e;
+  if (cols % 256 == 0) {
+    switch (cols / 256) {
+      case 1: return launch_ln_rows<1>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      case 2: return launch_ln_rows<2>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      case 4: return launch_ln_rows<4>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      case 8: return launch_ln_rows<8>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      case 12: return launch_ln_rows<12>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      case 16: return launch_ln_rows<16>(x, rows, shift, scale, codes, scales, gs_out, m_out, stats, amax, s);
+      default: break;
+    }
+  }
+  // generic widths: row loop per lane, then one thread per 16-element block
   const int64_t blocks = (rows + 7) / 8;
   ln_stats_amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), rows, cols,
                                                         reinterpret_cast<const uint16_t*>(shift),
