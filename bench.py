@@ -77,6 +77,26 @@ def stage_work(wl):
     }
 
 
+def committed_traffic(wl, stage):
+    """DRAM bytes per launch of a stage's kernel from the committed ncu capture
+    (profiles/dram_traffic_<workload>.json), or None when there is none or the
+    kernel source changed since it was taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"dram_traffic_{wl.name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(stage)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "diffusion_transformer_image_nvfp4_b200", "csrc", ent["source"])
+    if not os.path.exists(src) or hashlib.sha1(open(src, "rb").read()).hexdigest() != ent["sha1"]:
+        return None
+    return ent["bytes"]
+
+
 def tensor_peak_key(clk):
     """Burst bf16 peak when the timed region ran at full clock (no power cap
     pulled the SM clock down), the sustained one otherwise."""
@@ -395,7 +415,7 @@ def run_ours(args, wl):
     dom = max(stages, key=lambda s: stages[s]["ms"])
     roof = {k: stages[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac")}
     roof["kernel"] = dom
-    roof["traffic"] = None
+    roof["traffic"] = committed_traffic(wl, dom)
     kind = "burst" if pk == "bf16_tflops" else "sustained"
     roof["peak_source"] = (f"{peaks['source']} ({kind} bf16 x nominal dense ratio)" if roof["bound"] == "tensor"
                            else f"{peaks['source']} (copy)")
