@@ -48,7 +48,7 @@ class _NVFP4Tensor(ctypes.Structure):
 class _Epilogue(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("out_dtype", ctypes.c_int), ("out", ctypes.c_void_p),
                 ("rope_cs", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("residual", ctypes.c_void_p),
-                ("amax_out", ctypes.c_void_p)]
+                ("amax_out", ctypes.c_void_p), ("tile", ctypes.c_int)]
 
 
 class _TokenLayout(ctypes.Structure):
@@ -213,9 +213,14 @@ def ln_modulate_quantize_nvfp4_static(x, shift, scale, export_m=False):
     return (q, m) if export_m else q
 
 
+GEMM_TILES = {"auto": 0, "1cta_128x128": 1, "1cta_128x256": 2, "2sm_256x128": 3, "2sm_256x256": 4}
+
+
 def gemm_nvfp4_fused(A, W, epilogue="none", out=None, out_dtype=torch.bfloat16, rope_cs=None, gate=None,
-                     residual=None, amax=None):
-    """kl_gemm_nvfp4_fused: C = gA gW dec(A) dec(W)^T with a fused epilogue."""
+                     residual=None, amax=None, tile="auto"):
+    """kl_gemm_nvfp4_fused: C = gA gW dec(A) dec(W)^T with a fused epilogue.
+
+    tile: "auto" or one of GEMM_TILES (forces an output-tile variant)."""
     if A.layout != "mma" or W.layout != "mma" or A.cols != W.cols:
         raise ValueError("operands must share K and use the MMA scale layout")
     M, N, K = A.rows, W.rows, A.cols
@@ -224,7 +229,7 @@ def gemm_nvfp4_fused(A, W, epilogue="none", out=None, out_dtype=torch.bfloat16, 
         cols = N // 2 if kind == EPI["swiglu"] else N
         out = torch.empty((M, cols), dtype=out_dtype, device=A.codes.device)
     epi = _Epilogue(kind, KL_OUT_F32 if out.dtype == torch.float32 else KL_OUT_BF16, out.data_ptr(), _ptr(rope_cs),
-                    _ptr(gate), _ptr(residual), _ptr(amax))
+                    _ptr(gate), _ptr(residual), _ptr(amax), GEMM_TILES[tile])
     a, w = A.abi(), W.abi()
     _check(lib().kl_gemm_nvfp4_fused(ctypes.byref(a), ctypes.byref(w), M, N, K, ctypes.byref(epi), _stream()),
            "kl_gemm_nvfp4_fused")

@@ -71,12 +71,31 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle swz = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapSwizzle swz = swizzle_bytes == 64    ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : swizzle_bytes == 0   ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                                        : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return false;
+  }
+  return true;
+}
+
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
+                  const uint64_t strides_bytes[2], const uint32_t box[3]) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled (3D) failed (%d)", (int)r);
     return false;
   }
   return true;
@@ -233,7 +252,10 @@ kl_status kl_gemm_nvfp4_fused(const kl_nvfp4_tensor* A, const kl_nvfp4_tensor* W
   g.gate = epi->gate;
   g.residual = epi->residual;
   g.amax = epi->amax_out;
-  g.force_bn = 0;
+  static const int kTileBn[5] = {0, 128, 256, 384, 512};
+  if (epi->tile < KL_TILE_AUTO || epi->tile > KL_TILE_2SM_256x256) return KL_ERR_INVALID_ARG;
+  if ((epi->tile == KL_TILE_1CTA_128x256 || epi->tile == KL_TILE_2SM_256x256) && N % 256) return KL_ERR_UNSUPPORTED_SHAPE;
+  g.force_bn = kTileBn[epi->tile];
   cudaError_t e = launch_gemm_nvfp4(g, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KL_OK : cuda_fail(e);
 }

@@ -76,24 +76,50 @@ struct GemmCfg {
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 };
 
+// 32 bf16 (64 bytes) of one row.  Each thread of a warp writes a different
+// row, so one store instruction touches 32 rows: 32-byte stores (dst 32-byte
+// aligned) fill whole L2 sectors and halve the store instructions.
 __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
+  uint32_t w[16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    d[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  if ((reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 16 * h), "r"(w[8 * h]),
+                   "r"(w[8 * h + 1]), "r"(w[8 * h + 2]), "r"(w[8 * h + 3]), "r"(w[8 * h + 4]), "r"(w[8 * h + 5]),
+                   "r"(w[8 * h + 6]), "r"(w[8 * h + 7])
+                   : "memory");
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
 }
 __device__ __forceinline__ void load_bf16x32(const uint16_t* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint32_t u[16];
+  if ((reinterpret_cast<uintptr_t>(src) & 31) == 0) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w = __ldg(s + q);
-    uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    for (int h = 0; h < 2; ++h)
+      asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(u[8 * h]), "=r"(u[8 * h + 1]), "=r"(u[8 * h + 2]), "=r"(u[8 * h + 3]), "=r"(u[8 * h + 4]),
+                     "=r"(u[8 * h + 5]), "=r"(u[8 * h + 6]), "=r"(u[8 * h + 7])
+                   : "l"(src + 16 * h));
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[8 * q + 2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
-      v[8 * q + 2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w = __ldg(s + q);
+      u[4 * q] = w.x;
+      u[4 * q + 1] = w.y;
+      u[4 * q + 2] = w.z;
+      u[4 * q + 3] = w.w;
     }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    v[2 * j] = bf16_bits_to_f32(u[j] & 0xFFFFu);
+    v[2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
   }
 }
 // round to bf16 in place (the stored value), returning max |.|
@@ -105,6 +131,125 @@ __device__ __forceinline__ float round_bf16x32(float (&v)[32]) {
     m = fmaxf(m, fabsf(v[i]));
   }
   return m;
+}
+
+// Fused epilogue of one thread's accumulator slice: v holds BN/2 fp32
+// columns of one output row (SwiGLU: BN/4 gate then BN/4 up columns), already
+// drained from TMEM.  row / valid: the output row and whether it is < M; n0:
+// first column of the tile; half: which half of the tile's columns.
+template <int BN>
+__device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[BN / 2], float alpha, int64_t row,
+                                               bool valid, int64_t n0, int half, int lane) {
+  constexpr int HALF = BN / 2;
+  const int64_t D = p.N / 3;  // QKV only
+  const int H = (int)(D >> 7);
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) v[i] *= alpha;
+
+  if (p.epi == KL_EPI_SWIGLU) {
+    const int64_t F = p.N >> 1;
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < BN / 4; c += 32) {
+      float h[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        // silu(g) * u with the fast exp / divide intrinsics (relative
+        // error ~1e-6, far below the bf16 rounding of h); the argument
+        // is clamped so the denominator stays finite
+        const float gg = v[c + i], uu = v[BN / 4 + c + i];
+        h[i] = __fdividef(gg, 1.0f + __expf(fminf(-gg, 80.0f))) * uu;
+      }
+      amax = fmaxf(amax, round_bf16x32(h));
+      if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + half * (BN / 4) + c, h);
+    }
+    amax = warp_max(valid ? amax : 0.f);
+    if (lane == 0) atomic_max_nonneg(p.amax, amax);
+  } else {
+    // QKV: a thread's HALF (<= 128) columns lie in one head of one region
+    // (heads are 128 columns, n0 + half*HALF is a multiple of HALF)
+    float qkv_amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < HALF; c += 32) {
+      float* w = v + c;
+      const int64_t n = n0 + half * HALF + c;
+      if (p.epi == KL_EPI_NONE) {
+        if (valid) {
+          if (p.out_f32) {
+            float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.N + n);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) d[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          } else {
+            store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
+          }
+        }
+      } else if (p.epi == KL_EPI_GATED_RESIDUAL) {
+        if (valid) {
+          float gt[32], rs[32];
+          load_bf16x32(p.gate + n, gt);
+          load_bf16x32(p.residual + row * p.N + n, rs);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __fmaf_rn(gt[i], w[i], rs[i]);
+          store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
+        }
+      } else {  // KL_EPI_QKV_ROPE
+        const int region = (int)(n / D);
+        const int64_t cc = n - (int64_t)region * D;
+        const int head = (int)(cc >> 7);
+        if (region < 2) {
+          const int j0 = (int)((cc & 127) >> 1);
+          const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (valid ? row : 0) * 64 + j0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 t = __ldg(cs + q);  // (c, s) of two consecutive pairs
+            const float a0 = w[4 * q], b0 = w[4 * q + 1], a1 = w[4 * q + 2], b1 = w[4 * q + 3];
+            w[4 * q] = a0 * t.x - b0 * t.y;
+            w[4 * q + 1] = a0 * t.y + b0 * t.x;
+            w[4 * q + 2] = a1 * t.z - b1 * t.w;
+            w[4 * q + 3] = a1 * t.w + b1 * t.z;
+          }
+        }
+        qkv_amax = fmaxf(qkv_amax, round_bf16x32(*reinterpret_cast<float(*)[32]>(w)));
+        if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
+      }
+    }
+    if (p.epi == KL_EPI_QKV_ROPE) {
+      const int64_t nq = n0 + half * HALF;
+      const int region = (int)(nq / D);
+      const int head = (int)((nq - (int64_t)region * D) >> 7);
+      qkv_amax = warp_max(valid ? qkv_amax : 0.f);
+      if (lane == 0) atomic_max_nonneg(p.amax + region * H + head, qkv_amax);
+    }
+  }
+
+}
+
+// Drains one thread's slice of a 128 x BN accumulator (its TMEM lane group
+// at tbase) into registers: the BN/2 columns of tile half `half`, or for
+// SwiGLU the BN/4 gate and BN/4 up columns of the outputs that half owns.
+template <int BN>
+__device__ __forceinline__ void epilogue_drain(const GemmParams& p, uint32_t tbase, int half, float (&v)[BN / 2]) {
+  constexpr int HALF = BN / 2;
+  if constexpr (BN == 256) {
+    // columns [128*half, 128*half + 128): for SwiGLU that is exactly one
+    // 64-gate + 64-up row group, already in the order used by the epilogue
+    tmem_ld128(tbase + half * 128, v);
+  } else {
+    if (p.epi == KL_EPI_SWIGLU) {
+      // this thread's outputs o in [half*BN/4, (half+1)*BN/4): gate column
+      // (o/64)*128 + o%64 of the tile, up column = gate column + 64
+#pragma unroll
+      for (int c = 0; c < BN / 4; c += 32) {
+        const int o0 = half * (BN / 4) + c;
+        const int gcol = (o0 >> 6) * 128 + (o0 & 63);
+        tmem_ld32(tbase + gcol, *reinterpret_cast<float(*)[32]>(v + c));
+        tmem_ld32(tbase + gcol + 64, *reinterpret_cast<float(*)[32]>(v + BN / 4 + c));
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < HALF; c += 32) tmem_ld32(tbase + half * HALF + c, *reinterpret_cast<float(*)[32]>(v + c));
+    }
+  }
 }
 
 template <int BN, int KS>
@@ -152,20 +297,28 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Shared-memory descriptors of stage 0; a stage or K-step offset is added
+  // in 16-byte units to the start-address field (no carry: smem < 256 KB).
+  const uint64_t desc_a0 = smem_desc(smem_u32(smem), 16, C::SBO, C::LAYOUT);
+  const uint64_t desc_b0 = smem_desc(smem_u32(smem + C::A_BYTES), 16, C::SBO, C::LAYOUT);
+  const uint64_t desc_sf0 = smem_desc(smem_u32(smem + C::A_BYTES + C::B_BYTES), 0, 128, kLayoutNone);
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int64_t issued = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int mb = tile % p.num_m, nb = tile / p.num_m;
-        for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      const uint8_t* sfa_src = p.sfa + (int64_t)mb * p.kbn * 512;
+      const uint8_t* sfb_src = p.sfb + (int64_t)nb * (BN / 128) * p.kbn * 512;
+      for (int kt = 0; kt < p.num_kt; ++kt) {
+        if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
           uint8_t* ssfa = sb + C::B_BYTES;
@@ -175,115 +328,123 @@ __global__ void __launch_bounds__(352, 1)
           mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + sf_bytes * (1 + BN / 128));
           tma_load_2d(sa, &tmap_a, kt * C::ROWB, mb * 128, &full[stage]);
           tma_load_2d(sb, &tmap_b, kt * C::ROWB, nb * BN, &full[stage]);
-          bulk_load(ssfa, p.sfa + ((int64_t)mb * p.kbn + kt * KS) * 512, sf_bytes, &full[stage]);
+          bulk_load(ssfa, sfa_src + kt * (KS * 512), sf_bytes, &full[stage]);
 #pragma unroll
           for (int j = 0; j < BN / 128; ++j)
-            bulk_load(ssfb + j * KS * 512, p.sfb + ((int64_t)(nb * (BN / 128) + j) * p.kbn + kt * KS) * 512,
-                      sf_bytes, &full[stage]);
-          ++issued;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+            bulk_load(ssfb + j * KS * 512, sfb_src + (int64_t)j * p.kbn * 512 + kt * (KS * 512), sf_bytes,
+                      &full[stage]);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      if (!ok) {
-        // let every load already issued land before the CTA can exit
-        const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
-        for (int64_t i = first; i < issued; ++i) {
-          volatile int no_abort = 0;
-          mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), &no_abort);
-        }
+    }
+    if (!ok && lane == 0) {
+      // let every load already issued land before the CTA can exit
+      const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int64_t i = first; i < issued; ++i) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), &no_abort);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_nvf4(128, BN);
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+    constexpr uint32_t idesc = idesc_nvf4(128, BN);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      if (!warp_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+      for (int kt = 0; kt < p.num_kt; ++kt) {
+        // the operand tiles have landed and the scale-copy warp has moved
+        // this stage's block scales into the stage's TMEM scale buffer
+        if (!warp_wait(&full[stage], phase, abort_flag) || !warp_wait(&sf_ready[stage], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
-        for (int kt = 0; kt < p.num_kt; ++kt) {
-          // the operand tiles have landed and the scale-copy warp has moved
-          // this stage's block scales into the stage's TMEM scale buffer
-          if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_ready[stage], phase, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* sa = smem + stage * C::STAGE_BYTES;
-          const uint8_t* sb = sa + C::A_BYTES;
+        if (elect_one()) {
           const int nk = min(KS, p.kbn - kt * KS);
+          const uint64_t soff = (uint64_t)((stage * C::STAGE_BYTES) >> 4);
           const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4 * KS;
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t ad = smem_desc(smem_u32(sa + kk * 32), 16, C::SBO, C::LAYOUT);
-            const uint64_t bd = smem_desc(smem_u32(sb + kk * 32), 16, C::SBO, C::LAYOUT);
-            mma_nvf4(d_tmem, ad, bd, idesc, sfa_t + kk * 4, sfb_t + kk * (BN / 32), (kt | kk) != 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            if (kk < nk)
+              mma_nvf4(d_tmem, desc_a0 + soff + (uint64_t)(kk * 2), desc_b0 + soff + (uint64_t)(kk * 2), idesc,
+                       sfa_t + kk * 4, sfb_t + kk * (BN / 32), (kt | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        if (!ok) break;
-        tc_commit(&tfull[acc]);
-        if (++acc == C::ACC) {
-          acc = 0;
-          acc_phase ^= 1u;
+        __syncwarp();
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      // every MMA issued by this thread has completed before TMEM is freed
-      tc_commit(&drain[0]);
-      volatile int no_abort = 0;
-      mbar_wait(&drain[0], 0, &no_abort);
+      if (!ok) break;
+      if (elect_one()) tc_commit(&tfull[acc]);
+      __syncwarp();
+      if (++acc == C::ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
+    // every MMA issued by this warp has completed before TMEM is freed
+    if (elect_one()) tc_commit(&drain[0]);
+    __syncwarp();
+    volatile int no_abort = 0;
+    warp_wait(&drain[0], 0, &no_abort);
   } else if (warp == 10) {
     // -------------------------------------------------------- scale copier
     // Moves each stage's block scales from smem into that stage's TMEM scale
     // buffer as soon as the stage lands, ahead of the MMA issuer, so the MMA
-    // thread issues only MMAs.  A stage (and its scale buffer) is refilled
+    // warp issues only MMAs.  A stage (and its scale buffer) is refilled
     // only after the MMAs that read it have completed (empty -> producer ->
     // full), so the copies never overwrite scales still in use.
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* ssfa = smem + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-          const uint8_t* ssfb = ssfa + C::SFA_BYTES;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < p.num_kt; ++kt) {
+        if (!warp_wait(&full[stage], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
           const int nk = min(KS, p.kbn - kt * KS);
+          const uint64_t soff = (uint64_t)((stage * C::STAGE_BYTES) >> 4);
           const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4 * KS;
-          for (int kk = 0; kk < nk; ++kk) {
-            tmem_cp_32x128b_x4(sfa_t + kk * 4, smem_desc(smem_u32(ssfa + kk * 512), 0, 128, kLayoutNone));
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              tmem_cp_32x128b_x4(sfb_t + kk * (BN / 32) + j * 4,
-                                 smem_desc(smem_u32(ssfb + j * KS * 512 + kk * 512), 0, 128, kLayoutNone));
+          for (int kk = 0; kk < KS; ++kk) {
+            if (kk < nk) {
+              tmem_cp_32x128b_x4(sfa_t + kk * 4, desc_sf0 + soff + (uint64_t)(kk * 32));
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tmem_cp_32x128b_x4(sfb_t + kk * (BN / 32) + j * 4,
+                                   desc_sf0 + soff + (uint64_t)((C::SFA_BYTES + j * KS * 512 + kk * 512) >> 4));
+            }
           }
           tc_commit(&sf_ready[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      tc_commit(&drain[1]);
-      volatile int no_abort = 0;
-      mbar_wait(&drain[1], 0, &no_abort);
     }
+    if (elect_one()) tc_commit(&drain[1]);
+    __syncwarp();
+    volatile int no_abort = 0;
+    warp_wait(&drain[1], 0, &no_abort);
   } else {
     // ------------------------------------------------------------ epilogue
     // 8 warps: warp w reads TMEM lanes 32*(w%4).. (its rows) and one half of
@@ -295,8 +456,6 @@ __global__ void __launch_bounds__(352, 1)
     const int half = (warp - 2) >> 2;
     const int row_in_tile = quad * 32 + lane;
     const float alpha = __fmul_rn(__ldg(p.gsa), __ldg(p.gsw));
-    const int64_t D = p.N / 3;           // QKV only
-    const int H = (int)(D >> 7);
     int acc = 0;
     uint32_t acc_phase = 0;
     float v[HALF];
@@ -308,24 +467,7 @@ __global__ void __launch_bounds__(352, 1)
       const bool valid = row < p.M;
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
       const int64_t n0 = (int64_t)nb * BN;
-      if constexpr (BN == 256) {
-        // columns [128*half, 128*half + 128): for SwiGLU that is exactly one
-        // 64-gate + 64-up row group, already in the order used below
-        tmem_ld128(tbase + half * 128, v);
-      } else if (p.epi == KL_EPI_SWIGLU) {
-        // this thread's outputs o in [half*BN/4, (half+1)*BN/4): gate column
-        // (o/64)*128 + o%64 of the tile, up column = gate column + 64
-#pragma unroll
-        for (int c = 0; c < BN / 4; c += 32) {
-          const int o0 = half * (BN / 4) + c;
-          const int gcol = (o0 >> 6) * 128 + (o0 & 63);
-          tmem_ld32(tbase + gcol, *reinterpret_cast<float(*)[32]>(v + c));
-          tmem_ld32(tbase + gcol + 64, *reinterpret_cast<float(*)[32]>(v + BN / 4 + c));
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < HALF; c += 32) tmem_ld32(tbase + half * HALF + c, *reinterpret_cast<float(*)[32]>(v + c));
-      }
+      epilogue_drain<BN>(p, tbase, half, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -333,76 +475,7 @@ __global__ void __launch_bounds__(352, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
-#pragma unroll
-      for (int i = 0; i < HALF; ++i) v[i] *= alpha;
-
-      if (p.epi == KL_EPI_SWIGLU) {
-        const int64_t F = p.N >> 1;
-        float amax = 0.f;
-#pragma unroll
-        for (int c = 0; c < BN / 4; c += 32) {
-          float h[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            // silu(g) * u with the fast exp / divide intrinsics (relative
-            // error ~1e-6, far below the bf16 rounding of h); the argument
-            // is clamped so the denominator stays finite
-            const float gg = v[c + i], uu = v[BN / 4 + c + i];
-            h[i] = __fdividef(gg, 1.0f + __expf(fminf(-gg, 80.0f))) * uu;
-          }
-          amax = fmaxf(amax, round_bf16x32(h));
-          if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * F + (n0 >> 1) + half * (BN / 4) + c, h);
-        }
-        amax = warp_max(valid ? amax : 0.f);
-        if (lane == 0) atomic_max_nonneg(p.amax, amax);
-      } else {
-#pragma unroll
-        for (int c = 0; c < HALF; c += 32) {
-          float* w = v + c;
-          const int64_t n = n0 + half * HALF + c;
-          if (p.epi == KL_EPI_NONE) {
-            if (valid) {
-              if (p.out_f32) {
-                float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.N + n);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) d[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-              } else {
-                store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
-              }
-            }
-          } else if (p.epi == KL_EPI_GATED_RESIDUAL) {
-            if (valid) {
-              float gt[32], rs[32];
-              load_bf16x32(p.gate + n, gt);
-              load_bf16x32(p.residual + row * p.N + n, rs);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) w[i] = __fmaf_rn(gt[i], w[i], rs[i]);
-              store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
-            }
-          } else {  // KL_EPI_QKV_ROPE
-            const int region = (int)(n / D);
-            const int64_t cc = n - (int64_t)region * D;
-            const int head = (int)(cc >> 7);
-            if (region < 2) {
-              const int j0 = (int)((cc & 127) >> 1);
-              const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (valid ? row : 0) * 64 + j0);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 t = __ldg(cs + q);  // (c, s) of two consecutive pairs
-                const float a0 = w[4 * q], b0 = w[4 * q + 1], a1 = w[4 * q + 2], b1 = w[4 * q + 3];
-                w[4 * q] = a0 * t.x - b0 * t.y;
-                w[4 * q + 1] = a0 * t.y + b0 * t.x;
-                w[4 * q + 2] = a1 * t.z - b1 * t.w;
-                w[4 * q + 3] = a1 * t.w + b1 * t.z;
-              }
-            }
-            float amax = round_bf16x32(*reinterpret_cast<float(*)[32]>(w));
-            if (valid) store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n, *reinterpret_cast<float(*)[32]>(w));
-            amax = warp_max(valid ? amax : 0.f);
-            if (lane == 0) atomic_max_nonneg(p.amax + region * H + head, amax);
-          }
-        }
-      }
+      epilogue_apply<BN>(p, v, alpha, row, valid, n0, half, lane);
     }
   }
 
@@ -412,6 +485,341 @@ __global__ void __launch_bounds__(352, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ----------------------------------------------------------------- 2-SM
+// A CTA pair (cluster of 2) computes a 256 x BN output tile with
+// tcgen05.mma.cta_group::2 (M = 256 across the pair): each CTA holds 128 rows
+// of A, its BN/2-row half of the W rows, its 128 x BN fp32 accumulator in
+// TMEM, and in smem the block scales of its A rows (SFA) and of all BN W rows
+// (SFB).  One MMA instruction covers 256 x BN x 64 and one scale copy fills
+// both CTAs' TMEM, so per FLOP the pair issues half the instructions of two
+// single-CTA tiles, and each CTA loads half of W per stage (38 KB stages at
+// BN 256: 5 in flight).  BN 256: one accumulator (256 + 5 x 48 scale columns
+// of TMEM); BN 128: two (2 x 128 + 7 x 32), so the epilogue of one tile
+// overlaps the MMAs of the next.
+//
+// Roles (whole warps; one elected lane issues): warp 0 of both CTAs loads its
+// operand tiles and scales with cta_group::2 tensor copies that signal the
+// leader's stage barrier; on the leader, warp 10 copies each stage's scales
+// into TMEM (tcgen05.cp.cta_group::2) and warp 1 issues the MMAs, multicasting
+// its commits to both CTAs' stage-empty and accumulator-full barriers; warps
+// 2-9 of both CTAs drain their accumulator and arrive on the leader's
+// accumulator-empty barrier.
+#ifndef KL_SF_IN_MMA
+#define KL_SF_IN_MMA 1
+#endif
+
+template <int BN>
+struct Gemm2Cfg {
+  static constexpr int A_BYTES = 128 * 128;
+  static constexpr int B_BYTES = (BN / 2) * 128;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES;
+  static constexpr int ACC = BN == 256 ? 1 : 2;
+  static constexpr uint32_t ACC_COLS = BN;
+  static constexpr uint32_t SF_COLS = 16 + 16 * (BN / 128);
+  static constexpr uint32_t SF_BASE = ACC * ACC_COLS;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
+  static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "smem budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(352, 1)
+    gemm_nvfp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                          const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                          const GemmParams p) {
+  using C = Gemm2Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* sf_ready = empty + C::STAGES;
+  uint64_t* tfull = sf_ready + C::STAGES;  // ACC
+  uint64_t* tempty = tfull + C::ACC;       // ACC (leader: 16 arrivals each)
+  uint64_t* drain = tempty + C::ACC;       // 2
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
+    }
+    for (int a = 0; a < C::ACC; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);
+    }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_sfa);
+    prefetch_tmap(&tmap_sfb);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+  const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
+  const int num_m2 = (int)((p.M + 255) / 256);
+  const int num_tiles = num_m2 * (int)(p.N / BN);
+  // stage-0 descriptors; offsets are added in 16-byte units
+  const uint64_t desc_a0 = smem_desc(smem_u32(smem), 16, 1024, kLayoutSw128);
+  const uint64_t desc_b0 = smem_desc(smem_u32(smem + C::A_BYTES), 16, 1024, kLayoutSw128);
+  const uint64_t desc_sf0 = smem_desc(smem_u32(smem + C::A_BYTES + C::B_BYTES), 0, 128, kLayoutNone);
+
+  if (warp == 0) {
+    // ------------------------------------------------- producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+      const int mb2 = tile % num_m2, nb = tile / num_m2;
+      for (int kt = 0; kt < p.num_kt; ++kt) {
+        if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          uint8_t* ssfa = sb + C::B_BYTES;
+          uint8_t* ssfb = ssfa + C::SFA_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const uint32_t fb = full_leader + (uint32_t)stage * 8u;
+          tma_load_2d_pair(sa, &tmap_a, kt * 128, mb2 * 256 + (int)rank * 128, fb);
+          tma_load_2d_pair(sb, &tmap_b, kt * 128, nb * BN + (int)rank * (BN / 2), fb);
+          tma_load_2d_pair(ssfa, &tmap_sfa, 0, (mb2 * 2 + (int)rank) * p.kbn + kt * 4, fb);
+          tma_load_3d_pair(ssfb, &tmap_sfb, 0, kt * 4, nb * (BN / 128), fb);
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------- MMA issuer (leader)
+    if (leader) {
+      constexpr uint32_t idesc = idesc_nvf4(256, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        if (!warp_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)acc * C::ACC_COLS;
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+#if KL_SF_IN_MMA
+          if (!warp_wait(&full[stage], phase, abort_flag)) {
+#else
+          if (!warp_wait(&full[stage], phase, abort_flag) || !warp_wait(&sf_ready[stage], phase, abort_flag)) {
+#endif
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const int nk = min(4, p.kbn - kt * 4);
+            const uint64_t soff = (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+            const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
+            const uint32_t sfb_t = sfa_t + 16;
+#if KL_SF_IN_MMA
+            // scale copies ahead of the MMAs that read them: tcgen05.cp then
+            // tcgen05.mma from one thread execute in issue order
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk) {
+                tmem_cp_32x128b_x4_pair(sfa_t + kk * 4, desc_sf0 + soff + (uint64_t)(kk * 32));
+#pragma unroll
+                for (int j = 0; j < BN / 128; ++j)
+                  tmem_cp_32x128b_x4_pair(sfb_t + kk * (BN / 32) + j * 4,
+                                          desc_sf0 + soff + (uint64_t)((C::SFA_BYTES + j * 2048 + kk * 512) >> 4));
+              }
+            }
+#endif
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk)
+                mma_nvf4_pair(d_tmem, desc_a0 + soff + (uint64_t)(kk * 2), desc_b0 + soff + (uint64_t)(kk * 2), idesc,
+                              sfa_t + kk * 4, sfb_t + kk * (BN / 32), (kt | kk) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_mc(&empty[stage], 3);
+          }
+          __syncwarp();
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (elect_one()) tc_commit_pair_mc(&tfull[acc], 3);
+        __syncwarp();
+        if (++acc == C::ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (elect_one()) tc_commit_pair(&drain[0]);
+      __syncwarp();
+      volatile int no_abort = 0;
+      warp_wait(&drain[0], 0, &no_abort);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------ scale copier (leader)
+    if (leader && !KL_SF_IN_MMA) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          if (!warp_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const int nk = min(4, p.kbn - kt * 4);
+            const uint64_t soff = (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+            const uint32_t sfa_t = tmem + C::SF_BASE + (uint32_t)stage * C::SF_COLS;
+            const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nk) {
+                tmem_cp_32x128b_x4_pair(sfa_t + kk * 4, desc_sf0 + soff + (uint64_t)(kk * 32));
+#pragma unroll
+                for (int j = 0; j < BN / 128; ++j)
+                  tmem_cp_32x128b_x4_pair(sfb_t + kk * (BN / 32) + j * 4,
+                                          desc_sf0 + soff + (uint64_t)((C::SFA_BYTES + j * 2048 + kk * 512) >> 4));
+              }
+            }
+            tc_commit_pair(&sf_ready[stage]);
+          }
+          __syncwarp();
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (elect_one()) tc_commit_pair(&drain[1]);
+      __syncwarp();
+      volatile int no_abort = 0;
+      warp_wait(&drain[1], 0, &no_abort);
+    }
+  } else {
+    // ---------------------------------------------- epilogue (both CTAs)
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row_in_tile = quad * 32 + lane;
+    const float alpha = __fmul_rn(__ldg(p.gsa), __ldg(p.gsw));
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    float v[BN / 2];
+    for (int tile = pair; tile < num_tiles; tile += npairs) {
+      const int mb2 = tile % num_m2, nb = tile / num_m2;
+      if (!warp_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)acc * C::ACC_COLS;
+      epilogue_drain<BN>(p, tb, half, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)acc * 8u);
+      if (++acc == C::ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      const int64_t row = (int64_t)mb2 * 256 + rank * 128 + row_in_tile;
+      epilogue_apply<BN>(p, v, alpha, row, row < p.M, (int64_t)nb * BN, half, lane);
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while its pair may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN>
+static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
+  using C = Gemm2Cfg<BN>;
+  CUtensorMap ta, tb, tsa, tsb;
+  const uint64_t kbn = (uint64_t)(a.K / 64);
+  // block scales: SFA as rows of one 512-byte atom (128 x uint32), 4 atoms
+  // (one K stage) per box; SFB as (atom, K block, 128-row block of W), a box
+  // of 4 K blocks x BN/128 row blocks
+  const uint64_t sfb_dims[3] = {128, kbn, (uint64_t)(a.N / 128)};
+  const uint64_t sfb_strides[2] = {512, kbn * 512};
+  const uint32_t sfb_box[3] = {128, 4, (uint32_t)(BN / 128)};
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, (uint64_t)(a.K / 2), (uint64_t)a.M,
+                    (uint64_t)(a.K / 2), 128, 128, 128) ||
+      !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                    (uint64_t)(a.K / 2), 128, BN / 2, 128) ||
+      !make_tmap_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.a_scales, 128, (uint64_t)((a.M + 127) / 128) * kbn, 512,
+                    128, 4, 0) ||
+      !make_tmap_3d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.w_scales, sfb_dims, sfb_strides, sfb_box))
+    return cudaErrorInvalidValue;
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.sfa = reinterpret_cast<const uint8_t*>(a.a_scales);
+  p.sfb = reinterpret_cast<const uint8_t*>(a.w_scales);
+  p.gsa = a.a_gs;
+  p.gsw = a.w_gs;
+  p.epi = a.epi;
+  p.out_f32 = a.out_f32;
+  p.out = a.out;
+  p.rope_cs = reinterpret_cast<const float2*>(a.rope_cs);
+  p.gate = reinterpret_cast<const uint16_t*>(a.gate);
+  p.residual = reinterpret_cast<const uint16_t*>(a.residual);
+  p.amax = a.amax;
+  p.num_m = (int)((a.M + 255) / 256);
+  p.num_tiles = p.num_m * (int)(a.N / BN);
+  p.kbn = (int)kbn;
+  p.num_kt = (p.kbn + 3) / 4;
+  cudaError_t e =
+      cudaFuncSetAttribute(gemm_nvfp4_2sm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int pairs_max = device_sm_count() / 2;
+  const int pairs = p.num_tiles < pairs_max ? p.num_tiles : pairs_max;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(352);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN>, ta, tb, tsa, tsb, p);
 }
 
 template <int BN, int KS>
@@ -456,10 +864,16 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
 #define KL_GEMM_KSTEPS 4
 #endif
 
+// Tile choice: 2-SM 256 x BN pair tiles when M > 128 (BN = 256 when
+// N % 256 == 0, else 128); otherwise one-CTA 128 x 256 or 128 x 128 tiles.
+// force_bn: 0 automatic, 512 / 384 pair tiles of width 256 / 128, 256 / 128
+// one-CTA tiles.
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   int bn = a.force_bn;
-  if (bn == 0) bn = (a.N % 256 == 0) ? 256 : 128;
-  if (bn == 256 && a.N % 256 != 0) return cudaErrorInvalidValue;
+  if (bn == 0) bn = a.M > 128 ? ((a.N % 256 == 0) ? 512 : 384) : ((a.N % 256 == 0) ? 256 : 128);
+  if ((bn == 256 || bn == 512) && a.N % 256 != 0) return cudaErrorInvalidValue;
+  if (bn == 512) return launch_2sm<256>(a, s);
+  if (bn == 384) return launch_2sm<128>(a, s);
   return bn == 256 ? launch_bn<256, KL_GEMM_KSTEPS>(a, s) : launch_bn<128, KL_GEMM_KSTEPS>(a, s);
 }
 

@@ -39,7 +39,7 @@ struct GemmArgs {
   const void* gate;
   const void* residual;
   float* amax;
-  int force_bn;   // 0 = heuristic, else 128 or 256
+  int force_bn;   // 0 = heuristic; 128 / 256 one-CTA tiles, 384 / 512 2-SM pair tiles 256 x 128 / 256 x 256
 };
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s);
 
@@ -60,8 +60,11 @@ struct AttnArgs {
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
 // tensor maps (kl_api.cu)
-// 2D tensor map, box_inner x box_outer elements, 128-byte (or 64-byte) swizzle
+// 2D tensor map, box_inner x box_outer elements; swizzle_bytes 128, 64 or 0 (none)
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes = 128);
+// 3D tensor map without swizzle: dims / box innermost first, strides of dims 1 and 2 in bytes
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
+                  const uint64_t strides_bytes[2], const uint32_t box[3]);
 
 }  // namespace kl

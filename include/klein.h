@@ -186,7 +186,19 @@ typedef struct kl_epilogue {
   const void* residual;   /* GATED_RESIDUAL: bf16 [M, N] (may alias nothing else written) */
   float* amax_out;        /* QKV_ROPE: [3*N/384] per (q|k|v, head) max|out|; SWIGLU: [1].
                              Max-accumulated as non-negative floats: caller zero-fills. */
+  int tile;               /* KL_TILE_AUTO (0), or a forced output-tile variant (tests, tuning) */
 } kl_epilogue;
+
+/* Output-tile variants of kl_gemm_nvfp4_fused.  AUTO: 2-SM pair tiles of
+ * 256 x 256 (N % 256 == 0) or 256 x 128 when M > 128, else one-CTA 128 x 256
+ * (N % 256 == 0) or 128 x 128.  Every variant computes the same sums in the
+ * same K order per output, so all give bit-identical results.  A 256-wide
+ * variant with N % 256 != 0 returns KL_ERR_UNSUPPORTED_SHAPE. */
+#define KL_TILE_AUTO 0
+#define KL_TILE_1CTA_128x128 1
+#define KL_TILE_1CTA_128x256 2
+#define KL_TILE_2SM_256x128 3
+#define KL_TILE_2SM_256x256 4
 
 /*
  * kl_gemm_nvfp4_fused -- C[M,N] = gA*gW * sum_k dec(A)[m,k] * dec(W)[n,k]

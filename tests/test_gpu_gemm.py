@@ -130,3 +130,49 @@ def test_swiglu_epilogue():
     assert np.all(d <= np.abs(ref) * 2 ** -6 + 1e-5 * np.abs(ref).max())
     assert np.mean(d == 0) > 0.97
     assert to_np(amax)[0] == np.abs(got).max()
+
+
+TILES = ["1cta_128x128", "1cta_128x256", "2sm_256x128", "2sm_256x256"]
+
+
+@pytest.mark.parametrize("tile", TILES)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 384, 320), (1, 128, 512), (333, 512, 1536),
+                                   (1000, 3072, 768), (257, 768, 64)])
+def test_gemm_tile_variants_match_oracle(tile, M, N, K):
+    # every forced output-tile variant, including 2-SM pair tiles over a
+    # ragged last pair (M = 257, 333, 1000) and a single-row M
+    a, w, A, W = _operands(M, N, K, seed=7 * M + N + K)
+    if tile.endswith("x256") and N % 256:
+        with pytest.raises(kl.KLError, match="UNSUPPORTED_SHAPE"):
+            kl.gemm_nvfp4_fused(A, W, out_dtype=torch.float32, tile=tile)
+        return
+    got = to_np(kl.gemm_nvfp4_fused(A, W, out_dtype=torch.float32, tile=tile))
+    ref = _ref(a, w)
+    assert np.all(np.abs(got - ref) <= 1e-5 * _bound(a, w) + 1e-30)
+    assert rel_l2(got, ref) <= 1e-5
+
+
+def test_gemm_tile_variants_bit_identical_with_epilogues():
+    # the tile variants accumulate every output over the same 64-wide K steps
+    # in the same order, so all four give the same bits, epilogues included
+    M, N, K = 333, 1536, 768
+    a, w, A, W = _operands(M, N, K, seed=91)
+    Wp = kl.quantize_nvfp4(w.cuda(), swiglu_interleave=True)
+    x = normal_bf16((M, N), 92).cuda()
+    gate = normal_bf16((N,), 93, 0.1).cuda()
+    lay = (13, 16, 20, 0)  # 13 + 320 = 333 tokens
+    cs = kl.rope_table(*lay)
+    outs = {}
+    for tile in TILES:
+        amax_q = torch.zeros(3 * (N // 384), dtype=torch.float32, device="cuda")
+        amax_s = torch.zeros(1, dtype=torch.float32, device="cuda")
+        outs[tile] = [
+            to_np(kl.gemm_nvfp4_fused(A, W, out_dtype=torch.float32, tile=tile)),
+            to_np(kl.gemm_nvfp4_fused(A, W, "gated_residual", gate=gate, residual=x, tile=tile)),
+            to_np(kl.gemm_nvfp4_fused(A, W, "qkv_rope", rope_cs=cs, amax=amax_q, tile=tile)),
+            to_np(kl.gemm_nvfp4_fused(A, Wp, "swiglu", amax=amax_s, tile=tile)),
+            to_np(amax_q), to_np(amax_s),
+        ]
+    for tile in TILES[1:]:
+        for got, want in zip(outs[tile], outs[TILES[0]]):
+            np.testing.assert_array_equal(got, want)
