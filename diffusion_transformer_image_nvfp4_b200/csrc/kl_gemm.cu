@@ -197,16 +197,16 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
         const int64_t cc = n - (int64_t)region * D;
         const int head = (int)(cc >> 7);
         if (region < 2) {
+          // the table is pair-major ([64, M] of (c, s)): the 32 lanes (32
+          // consecutive rows) read 256 contiguous bytes per pair
           const int j0 = (int)((cc & 127) >> 1);
-          const float4* cs = reinterpret_cast<const float4*>(p.rope_cs + (valid ? row : 0) * 64 + j0);
+          const float2* cs = p.rope_cs + (int64_t)j0 * p.M + (valid ? row : 0);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 t = __ldg(cs + q);  // (c, s) of two consecutive pairs
-            const float a0 = w[4 * q], b0 = w[4 * q + 1], a1 = w[4 * q + 2], b1 = w[4 * q + 3];
-            w[4 * q] = a0 * t.x - b0 * t.y;
-            w[4 * q + 1] = a0 * t.y + b0 * t.x;
-            w[4 * q + 2] = a1 * t.z - b1 * t.w;
-            w[4 * q + 3] = a1 * t.w + b1 * t.z;
+          for (int q = 0; q < 16; ++q) {
+            const float2 t = __ldg(cs + (int64_t)q * p.M);  // (c, s) of pair j0 + q
+            const float a0 = w[2 * q], b0 = w[2 * q + 1];
+            w[2 * q] = a0 * t.x - b0 * t.y;
+            w[2 * q + 1] = a0 * t.y + b0 * t.x;
           }
         }
         qkv_amax = fmaxf(qkv_amax, round_bf16x32(*reinterpret_cast<float(*)[32]>(w)));

@@ -406,11 +406,12 @@ __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restric
 // ------------------------------------------------------------ RoPE table
 __global__ void rope_table_kernel(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta,
                                   float2* __restrict__ cs) {
+  // pair-major: cs[j * T + t]
   const int64_t T = n_text + (1 + n_ref) * gh * gw;
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= T * 64) return;
-  const int64_t t = i >> 6;
-  const int j = (int)(i & 63);
+  const int j = (int)(i / T);
+  const int64_t t = i - (int64_t)j * T;
   double phi;
   if (t < n_text) {
     phi = (double)t * pow(theta, -2.0 * j / 128.0);
