@@ -15,13 +15,18 @@
 //    into TMEM; then O_t += P_t V_{j-1} (V read MN-major straight from its
 //    row-major tile) for the previous key tile, so the tensor core computes
 //    the next scores while the softmax warps exponentiate;
-//  * 4 softmax warps per query tile (thread = query row): one pass over the
-//    scores in registers; the running maximum m is only moved (and O, l
-//    rescaled in place -- O in TMEM after the previous P.V has landed) when a
-//    tile's maximum exceeds m by more than TAU (log2 units), so
-//    p = 2^(s*c - m) <= 2^TAU; p * P_SCALE is rounded to E4M3 (BF16: bf16)
-//    and written to a double-buffered smem P tile in the MMA's K-major
-//    swizzled layout; l sums the unrounded p * P_SCALE.
+//  * 8 softmax warps per query tile: two per 32-row TMEM lane group, each
+//    thread owning one query row and 64 of the 128 score columns (four
+//    softmax warps per SM sub-partition hide the exponent and conversion
+//    latencies).  Both halves of a row reduce the row maximum over all 128
+//    scores (the other half's columns are read from TMEM for that only), so
+//    they take the same decisions without exchanging anything; the running
+//    maximum m is only moved (and O, l rescaled in place -- O in TMEM after
+//    the previous P.V has landed) when a tile's maximum exceeds m by more
+//    than TAU (log2 units), so p = 2^(s*c - m) <= 2^TAU; p * P_SCALE is
+//    rounded to E4M3 (BF16: bf16) and written to a double-buffered smem P
+//    tile in the MMA's K-major swizzled layout; each half sums its unrounded
+//    p * P_SCALE, and the halves' sums are added once at the end.
 //    Finally O = O_tmem / l (FP8: times s_v), bf16, and a tensor amax.
 // TMEM per query tile: S [128 cols] + O [128 cols].
 #include "kl_common.cuh"
@@ -51,27 +56,60 @@ struct AttnCfg {
   static constexpr float TAU = FP8 ? 4.0f : 8.0f;  // lazy-rescale threshold, log2 units
   static constexpr float P_SCALE = FP8 ? 16.0f : 1.0f;  // p * P_SCALE <= 2^(TAU+4) <= 448
   static constexpr float LOG2_P_SCALE = FP8 ? 4.0f : 0.0f;
+  static constexpr int SPLIT = 2;                  // softmax warps per 32 query rows
+  static constexpr int COLS = 128 / SPLIT;         // score / output columns per softmax thread
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = QT * TILE;
   static constexpr int P_OFF = KV_OFF + NS * 2 * TILE;
   static constexpr int BAR_OFF = P_OFF + QT * 2 * TILE;
-  static constexpr int THREADS = 64 + QT * 128;
+  static constexpr int L_OFF = BAR_OFF + 512;      // partial row sums, QT x SPLIT x 128 fp32
+  static constexpr int SOFTMAX_THREADS = QT * 128 * SPLIT;
+  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr uint32_t TMEM_COLS = QT * 256;
-  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
+  static constexpr int SMEM_BYTES = L_OFF + QT * SPLIT * 128 * 4 + 1024;
   static_assert(SMEM_BYTES <= 232448, "smem budget");
 };
 
-// K-major SW128 descriptor of MMA step kk inside a [128 rows x 128 elems] tile
-template <bool FP8>
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
-  const uint32_t off = FP8 ? (uint32_t)kk * 32u : (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-  return smem_desc(base + off, 16, 1024, kLayoutSw128);
-}
-// MN-major SW128 descriptor of MMA step kk of a V tile [128 keys x 128 dims]
-template <bool FP8>
-__device__ __forceinline__ uint64_t vdesc(uint32_t base, int kk) {
-  const uint32_t rows_per_step = FP8 ? 32u : 16u;
-  return smem_desc(base + (uint32_t)kk * rows_per_step * 128u, 16384, 1024, kLayoutSw128);
+// Share of the softmax exponentials computed on the FMA pipe instead of the
+// MUFU unit: KL_ATTN_POLY of every 8 element pairs.  The MUFU unit issues a
+// quarter warp of ex2 per cycle per SM sub-partition, which alone would hold
+// the softmax to about half the FP8 tensor-core rate; running some of the
+// exponentials as FMAs keeps both pipes busy.
+#ifndef KL_ATTN_STAGGER
+#define KL_ATTN_STAGGER 0
+#endif
+#ifndef KL_ATTN_POLY
+#define KL_ATTN_POLY 0
+#endif
+
+// 2^x for two floats on the FMA pipe.  Cody-Waite style range reduction
+// x = j + f, j = rint(x) (the 1.5 * 2^23 add rounds to an integer), |f| <= 1/2;
+// 2^f by a degree-4 polynomial whose coefficients were fitted here to the
+// relative error of 2^f on [-1/2, 1/2] (Lawson-weighted least squares; max
+// relative error 2.9e-6 in fp32 Horner form, far below the E4M3 rounding of
+// p that follows); 2^j is added to the exponent field (j << 23).  x is
+// clamped to >= -125 so the exponent stays normal; 2^-125 rounds to 0 in
+// E4M3 like the exact value would.
+__device__ __forceinline__ uint64_t exp2_poly_f32x2(uint64_t x2) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float xl, xh;
+  unpack_f32x2(x2, xl, xh);
+  const uint64_t x = pack_f32x2(fmaxf(xl, -125.0f), fmaxf(xh, -125.0f));
+  const uint64_t t = add_f32x2(x, pack_f32x2(kRound, kRound));
+  const uint64_t jf = add_f32x2(t, pack_f32x2(-kRound, -kRound));
+  const uint64_t f = fma_f32x2(jf, pack_f32x2(-1.0f, -1.0f), x);
+  uint64_t q = fma_f32x2(pack_f32x2(0.009582853f, 0.009582853f), f, pack_f32x2(0.055906426f, 0.055906426f));
+  q = fma_f32x2(q, f, pack_f32x2(0.24024099f, 0.24024099f));
+  q = fma_f32x2(q, f, pack_f32x2(0.69312418f, 0.69312418f));
+  q = fma_f32x2(q, f, pack_f32x2(1.0f, 1.0f));
+  float ql, qh, tl, th;
+  unpack_f32x2(q, ql, qh);
+  unpack_f32x2(t, tl, th);
+  // bits(t) = bits(1.5 * 2^23) + j and bits(1.5 * 2^23) is a multiple of 2^9,
+  // so bits(t) << 23 == j << 23 (mod 2^32)
+  ql = __int_as_float(__float_as_int(ql) + (int)((uint32_t)__float_as_int(tl) << 23));
+  qh = __int_as_float(__float_as_int(qh) + (int)((uint32_t)__float_as_int(th) << 23));
+  return pack_f32x2(ql, qh);
 }
 
 template <bool FP8>
@@ -113,11 +151,11 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&s_empty[t], 4);
+      mbar_init(&s_empty[t], 4 * C::SPLIT);
       mbar_init(&o_done[t], 1);
       mbar_init(&o_last[t], 1);
       for (int b = 0; b < 2; ++b) {
-        mbar_init(&p_full[2 * t + b], 4);
+        mbar_init(&p_full[2 * t + b], 4 * C::SPLIT);
         mbar_init(&p_empty[2 * t + b], 1);
       }
     }
@@ -138,27 +176,34 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   uint8_t* p_smem = smem + C::P_OFF;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA
+    // -------------------------------------------------------------- TMA
+    // the whole warp runs the loop; one elected lane issues
+    if (elect_one()) {
       prefetch_tmap(&tq);
       prefetch_tmap(&tk);
       prefetch_tmap(&tv);
       mbar_arrive_expect_tx(q_full, QT * C::TILE);
       for (int t = 0; t < QT; ++t) tma_tile<FP8>(q_smem + t * C::TILE, &tq, h * 128, (qblk * QT + t) * 128, q_full);
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % C::NS;
-        if (!mbar_wait(&kv_empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
+    }
+    __syncwarp();
+    int issued = 0;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int s = j % C::NS;
+      if (!warp_wait(&kv_empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      if (elect_one()) {
         uint8_t* ks = kv_smem + s * 2 * C::TILE;
         mbar_arrive_expect_tx(&kv_full[s], 2 * C::TILE);
         tma_tile<FP8>(ks, &tk, h * 128, j * 128, &kv_full[s]);
         tma_tile<FP8>(ks + C::TILE, &tv, h * 128, j * 128, &kv_full[s]);
-        ++issued;
       }
+      __syncwarp();
+      ++issued;
+    }
+    if (lane == 0) {
       volatile int no_abort = 0;
       mbar_wait(q_full, 0, &no_abort);
       if (!ok) {
@@ -170,106 +215,138 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA
-      const uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
-      const uint32_t id_pv = FP8 ? idesc_e4m3(128, 128, 1) : idesc_bf16(128, 128, 1);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int j = 0; ok && j <= n; ++j) {
+    // -------------------------------------------------------------- MMA
+    // The whole warp runs the loop and one elected lane issues; smem
+    // descriptors are built once and advanced by adding offsets (16-byte
+    // units) to the start-address field.
+    constexpr uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
+    constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, 128, 1) : idesc_bf16(128, 128, 1);
+    constexpr uint64_t TILE16 = (uint64_t)(C::TILE >> 4);
+    const uint64_t q_desc0 = smem_desc(smem_u32(q_smem), 16, 1024, kLayoutSw128);
+    const uint64_t k_desc0 = smem_desc(smem_u32(kv_smem), 16, 1024, kLayoutSw128);
+    const uint64_t v_desc0 = smem_desc(smem_u32(kv_smem + C::TILE), 16384, 1024, kLayoutSw128);
+    const uint64_t p_desc0 = smem_desc(smem_u32(p_smem), 16, 1024, kLayoutSw128);
+    bool ok = warp_wait(q_full, 0, abort_flag);
+    // Issue order per key tile j: for each query tile t, S_t(j) = Q_t K_j^T
+    // then O_t += P_t(j-1) V_{j-1}.
+    for (int j = 0; ok && j <= n; ++j) {
+      const int s = j % C::NS;
+      if (j < n && !warp_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const int jj = j - 1, sp = (jj + C::NS) % C::NS, b = jj & 1;
+      const uint64_t k_desc = k_desc0 + (uint64_t)(2 * s) * TILE16;
+      const uint64_t v_desc = v_desc0 + (uint64_t)(2 * sp) * TILE16;
+      for (int t = 0; t < QT && ok; ++t) {
         if (j < n) {
-          const int s = j % C::NS;
-          if (!mbar_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag)) {
+          if (!warp_wait(&s_empty[t], ((uint32_t)j & 1u) ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t k_addr = smem_u32(kv_smem + s * 2 * C::TILE);
-          for (int t = 0; t < QT && ok; ++t) {
-            if (!mbar_wait(&s_empty[t], ((uint32_t)j & 1u) ^ 1u, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t q_addr = smem_u32(q_smem + t * C::TILE);
+          tc_fence_after();
+          if (elect_one()) {
+            const uint64_t q_desc = q_desc0 + (uint64_t)t * TILE16;
 #pragma unroll
             for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              const uint64_t ad = kmajor_desc<FP8>(q_addr, kk), bd = kmajor_desc<FP8>(k_addr, kk);
+              // K-major step kk: FP8 32 bytes, BF16 16 elements (64-element halves 16 KB apart)
+              const uint64_t off = FP8 ? (uint64_t)(kk * 2) : (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
               if (FP8)
-                mma_f8(tmem + t * 256, ad, bd, id_qk, kk > 0);
+                mma_f8(tmem + t * 256, q_desc + off, k_desc + off, id_qk, kk > 0);
               else
-                mma_f16(tmem + t * 256, ad, bd, id_qk, kk > 0);
+                mma_f16(tmem + t * 256, q_desc + off, k_desc + off, id_qk, kk > 0);
             }
             tc_commit(&s_full[t]);
           }
-          if (!ok) break;
+          __syncwarp();
         }
         if (j >= 1) {
-          const int jj = j - 1, s = jj % C::NS, b = jj & 1;
-          const uint32_t v_addr = smem_u32(kv_smem + s * 2 * C::TILE + C::TILE);
-          for (int t = 0; t < QT && ok; ++t) {
-            if (!mbar_wait(&p_full[2 * t + b], (uint32_t)(jj >> 1) & 1u, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t p_addr = smem_u32(p_smem + (2 * t + b) * C::TILE);
+          if (!warp_wait(&p_full[2 * t + b], (uint32_t)(jj >> 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint64_t p_desc = p_desc0 + (uint64_t)(2 * t + b) * TILE16;
 #pragma unroll
             for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              const uint64_t ad = kmajor_desc<FP8>(p_addr, kk), bd = vdesc<FP8>(v_addr, kk);
+              const uint64_t off = FP8 ? (uint64_t)(kk * 2) : (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+              // MN-major V: step kk covers keys [kk*R, kk*R + R), R = 32 (FP8) / 16 (BF16) rows of 128 B
+              const uint64_t voff = (uint64_t)(kk * (FP8 ? 32 : 16) * 8);
               if (FP8)
-                mma_f8(tmem + t * 256 + 128, ad, bd, id_pv, (jj | kk) != 0);
+                mma_f8(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (jj | kk) != 0);
               else
-                mma_f16(tmem + t * 256 + 128, ad, bd, id_pv, (jj | kk) != 0);
+                mma_f16(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (jj | kk) != 0);
             }
             tc_commit(&o_done[t]);
             tc_commit(&p_empty[2 * t + b]);
             if (jj == n - 1) tc_commit(&o_last[t]);
           }
-          if (!ok) break;
-          tc_commit(&kv_empty[s]);
+          __syncwarp();
         }
       }
-      tc_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort);
+      if (!ok) break;
+      // K/V stage of tile j-1 is free once the last P.V that reads it is done
+      if (j >= 1) {
+        if (elect_one()) tc_commit(&kv_empty[sp]);
+        __syncwarp();
+      }
     }
+    if (elect_one()) tc_commit(drain);
+    __syncwarp();
+    volatile int no_abort = 0;
+    warp_wait(drain, 0, &no_abort);
   } else {
     // ------------------------------------------------------------ softmax
-    const int sw = warp - 2;              // softmax warp 0 .. 4*QT-1
-    const int t = sw >> 2;                // query tile of this warp
+    constexpr int COLS = C::COLS;
+    const int g = (warp - 2) >> 2;        // 4 consecutive warps cover the 4 lane groups
+    const int t = g / C::SPLIT;           // query tile of this warp
+    const int part = g % C::SPLIT;        // its score / output columns [part*COLS, +COLS)
     const int quad = warp & 3;            // TMEM lane group this warp may access
     const int r = quad * 32 + lane;       // query row inside the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(t * 256);
-    const uint32_t s_tmem = lane_base, o_tmem = lane_base + 128;
+    const uint32_t s_tmem = lane_base, o_tmem = lane_base + 128 + (uint32_t)(part * COLS);
     float c = p.c_log2;
     if (FP8) c *= __ldg(p.sq + h) * __ldg(p.sk + h);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+#if KL_ATTN_STAGGER
+    if (t == 1) {
+      const long long t0 = clock64();
+      while (clock64() - t0 < KL_ATTN_STAGGER) {
+      }
+    }
+#endif
     for (int j = 0; j < n; ++j) {
       if (!warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sc[128];
+      const int64_t rem = p.T - (int64_t)j * 128;
+      float sc[COLS];
+      float mk[8];
+      // row maximum over all 128 scores: first the other half's columns
+      // (read for the maximum only), then this thread's own, kept in sc
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(s_tmem + cc * 32, *reinterpret_cast<float(*)[32]>(sc + cc * 32));
+      for (int k = 0; k < 8; ++k) mk[k] = -INFINITY;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int col0 = pass == 0 ? (1 - part) * COLS : part * COLS;
+        tmem_ld64(s_tmem + col0, sc);
+        if (rem < 128) {
+#pragma unroll
+          for (int i = 0; i < COLS; ++i)
+            if (col0 + i >= rem) sc[i] = -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < COLS; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], sc[i + 2 * k], sc[i + 2 * k + 1]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[t]);
-      const int64_t rem = p.T - (int64_t)j * 128;
-      if (rem < 128) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= rem) sc[i] = -INFINITY;
-      }
-      // row maximum: 8 independent chains of 3-input max
-      float mk[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mk[k] = fmaxf(sc[2 * k], sc[2 * k + 1]);
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], sc[i + 2 * k], sc[i + 2 * k + 1]);
       float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7])) * c;
       // this P buffer was last read by P.V of key tile j-2: once it is free,
       // every P.V up to j-2 has landed
@@ -281,9 +358,9 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       const bool move = mx > m + C::TAU;
       if (__any_sync(0xffffffffu, move)) {
         // move the reference maximum of the rows that need it and rescale
-        // their O (in TMEM, after P.V of tile j-1 has landed) and l by
-        // 2^(m_old - m_new).  TMEM loads/stores are warp-wide, so the whole
-        // warp takes this path; rows that do not move use a factor of 1.
+        // their O columns (in TMEM, after P.V of tile j-1 has landed) and l
+        // by 2^(m_old - m_new).  TMEM loads/stores are warp-wide, so the
+        // whole warp takes this path; rows that do not move use a factor of 1.
         const float alpha = move ? ex2_approx(m - mx) : 1.0f;
         if (j > 0) {
           if (!warp_wait(&o_done[t], (uint32_t)(j - 1) & 1u, abort_flag)) {
@@ -292,7 +369,7 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < COLS / 32; ++cc) {
             float o[32];
             tmem_ld32(o_tmem + cc * 32, o);
 #pragma unroll
@@ -312,11 +389,16 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       const uint64_t mb2 = pack_f32x2(mb, mb);
       uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        float lo, hi;
-        unpack_f32x2(fma_f32x2(pack_f32x2(sc[i], sc[i + 1]), c2, mb2), lo, hi);
-        sc[i] = ex2_approx(lo);
-        sc[i + 1] = ex2_approx(hi);
+      for (int i = 0; i < COLS; i += 2) {
+        const uint64_t x2 = fma_f32x2(pack_f32x2(sc[i], sc[i + 1]), c2, mb2);
+        if (((i >> 1) & 7) < KL_ATTN_POLY) {
+          unpack_f32x2(exp2_poly_f32x2(x2), sc[i], sc[i + 1]);
+        } else {
+          float lo, hi;
+          unpack_f32x2(x2, lo, hi);
+          sc[i] = ex2_approx(lo);
+          sc[i + 1] = ex2_approx(hi);
+        }
         acc2[(i >> 1) & 3] = add_f32x2(acc2[(i >> 1) & 3], pack_f32x2(sc[i], sc[i + 1]));
       }
       float a0, a1, b0, b1;
@@ -324,23 +406,28 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       unpack_f32x2(add_f32x2(acc2[2], acc2[3]), b0, b1);
       const float rowsum = (a0 + a1) + (b0 + b1);
       if (FP8) {
+        // this thread's COLS bytes of the 128-byte P row: 16-byte chunks
+        // part*COLS/16 .., stored at chunk ^ (r & 7) (128-byte swizzle)
 #pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk) {
+        for (int chunk = 0; chunk < COLS / 16; ++chunk) {
           uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float* x = sc + chunk * 16 + q * 4;
             w[q] = f32x2_to_e4m3x2(x[0], x[1]) | (f32x2_to_e4m3x2(x[2], x[3]) << 16);
           }
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const int gc = part * (COLS / 16) + chunk;
+          *reinterpret_cast<uint4*>(prow + ((gc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
+        // bf16 P row: two 16 KB halves of 64 elements; 16-byte chunk gc
 #pragma unroll
-        for (int chunk = 0; chunk < 16; ++chunk) {
+        for (int chunk = 0; chunk < COLS / 8; ++chunk) {
           const float* x = sc + chunk * 8;
           const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                                      pack_bf16x2(x[6], x[7]));
-          *reinterpret_cast<uint4*>(prow + (chunk >> 3) * 16384 + (((chunk & 7) ^ (r & 7)) << 4)) = w;
+          const int gc = part * (COLS / 8) + chunk;
+          *reinterpret_cast<uint4*>(prow + (gc >> 3) * 16384 + (((gc & 7) ^ (r & 7)) << 4)) = w;
         }
       }
       l += rowsum;
@@ -348,19 +435,27 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
     }
+    // the row sum is the sum of the halves' partial sums; every softmax
+    // thread reaches this barrier (also after a failed wait)
+    float* lsm = reinterpret_cast<float*>(smem + C::L_OFF);
+    lsm[(t * C::SPLIT + part) * 128 + r] = l;
+    asm volatile("bar.sync 1, %0;" ::"n"(C::SOFTMAX_THREADS) : "memory");
+    float lsum = 0.f;
+#pragma unroll
+    for (int q = 0; q < C::SPLIT; ++q) lsum += lsm[(t * C::SPLIT + q) * 128 + r];
     // epilogue: O / l (FP8: times s_v), bf16, tensor amax
     ok = __all_sync(0xffffffffu, ok);
     if (ok) ok = warp_wait(&o_last[t], 0, abort_flag);
     const int64_t row = ((int64_t)qblk * QT + t) * 128 + r;
     const bool valid_row = ok && row < p.T;
-    float scale = 1.0f / l;  // l sums p * P_SCALE, so this also undoes P_SCALE
+    float scale = 1.0f / lsum;  // l sums p * P_SCALE, so this also undoes P_SCALE
     if (FP8) scale *= __ldg(p.sv + h);
     float amax = 0.f;
     if (ok) {
       tc_fence_after();
-      uint4* dst = reinterpret_cast<uint4*>(p.out + row * (int64_t)p.H * 128 + h * 128);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * (int64_t)p.H * 128 + h * 128 + part * COLS);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < COLS / 32; ++cc) {
         float o[32];
         tmem_ld32(o_tmem + cc * 32, o);
 #pragma unroll
