@@ -56,7 +56,10 @@ struct AttnCfg {
   static constexpr float TAU = FP8 ? 4.0f : 8.0f;  // lazy-rescale threshold, log2 units
   static constexpr float P_SCALE = FP8 ? 16.0f : 1.0f;  // p * P_SCALE <= 2^(TAU+4) <= 448
   static constexpr float LOG2_P_SCALE = FP8 ? 4.0f : 0.0f;
-  static constexpr int SPLIT = 2;                  // softmax warps per 32 query rows
+#ifndef KL_ATTN_SPLIT
+#define KL_ATTN_SPLIT 2
+#endif
+  static constexpr int SPLIT = KL_ATTN_SPLIT;     // softmax warps per 32 query rows (1 or 2)
   static constexpr int COLS = 128 / SPLIT;         // score / output columns per softmax thread
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = QT * TILE;
@@ -331,9 +334,12 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) mk[k] = -INFINITY;
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
+      for (int pass = C::SPLIT == 2 ? 0 : 1; pass < 2; ++pass) {
         const int col0 = pass == 0 ? (1 - part) * COLS : part * COLS;
-        tmem_ld64(s_tmem + col0, sc);
+        if constexpr (COLS == 128)
+          tmem_ld128(s_tmem + col0, sc);
+        else
+          tmem_ld64(s_tmem + col0, sc);
         if (rem < 128) {
 #pragma unroll
           for (int i = 0; i < COLS; ++i)
