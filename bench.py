@@ -186,6 +186,36 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+# ------------------------------------------------ multi-rank host logic
+# The same functions serve the NCCL run (device tensors) and the gloo CPU
+# tests of the N > 1 path.
+def rank_barrier(world, device=None):
+    """Barrier over the ranks (when there are several), then a device sync."""
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    if device is not None and device.type == "cuda":
+        torch.cuda.synchronize(device)
+
+
+def rank_max(v, world, device):
+    """max over ranks of a per-rank number (the job's time is its slowest rank)."""
+    if world == 1:
+        return float(v)
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, tokens_per_rank, steps, total_ms):
+    """Weak scaling: every rank runs its own image's block; the job processes
+    world * tokens_per_rank tokens per step in the slowest rank's time."""
+    return world * tokens_per_rank * steps / (total_ms * 1e-3)
+
+
 def config_of(wl, extra=None):
     c = {"workload": wl.name, "tokens": wl.n_tokens, "text_tokens": wl.n_text,
          "image_grid": f"{wl.grid_h}x{wl.grid_w}", "reference_images": wl.n_ref, "hidden": wl.hidden,
@@ -305,20 +335,10 @@ def run_ours(args, wl):
         raise SystemExit(f"device status after warm-up: {st}")
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.barrier()
-        torch.cuda.synchronize()
+        rank_barrier(world, dev)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        import torch.distributed as dist
-
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(v, world, dev)
 
     # value: the block captured once in a CUDA graph and replayed.  Every
     # step: L2 flush, then one replay bracketed by events on the stream.  The
@@ -357,7 +377,7 @@ def run_ours(args, wl):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms))
-    value = world * T * args.steps / (total_ms * 1e-3)
+    value = whole_job_value(world, T, args.steps, total_ms)
 
     # per-kernel breakdown: the same steps launched directly, with the
     # library recording an event between the stages of every step
@@ -437,7 +457,7 @@ def run_ours(args, wl):
             "attention_frac": round(work["attention"][1] / (stage_ms["attention"] * 1e-3) / 1e12 / att_peak, 4),
             "roofline": roof, "stages": stages, "gpu_launches": launches,
             "ms_per_step_direct_launch": round(eager_ms, 4),
-            "e2e": {"value": round(world * T * args.steps / (e2e_ms * 1e-3), 1), "unit": UNIT,
+            "e2e": {"value": round(whole_job_value(world, T, args.steps, e2e_ms), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
