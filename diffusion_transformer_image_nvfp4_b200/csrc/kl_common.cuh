@@ -393,9 +393,15 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) { return __ui
 __device__ __forceinline__ uint32_t f32_to_bf16_bits(float x) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
+// two floats -> two bf16 (RNE) in one word, lo in the low half; one cvt
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
+// a word of two bf16 -> the two floats (exact)
+__device__ __forceinline__ float bf16lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -419,6 +425,21 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// float pair from a word of two bf16
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) { return pack_f32x2(bf16lo_f32(w), bf16hi_f32(w)); }
+// max |.| of the bf16 values of two words, as a word of two bf16 magnitudes:
+// for non-negative bf16 the bit patterns order like the values
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t acc, uint32_t w) {
+  return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+__device__ __forceinline__ float bf16x2_hmax_f32(uint32_t w) {
+  return fmaxf(bf16lo_f32(w), bf16hi_f32(w));
 }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;

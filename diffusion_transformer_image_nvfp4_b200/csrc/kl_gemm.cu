@@ -195,7 +195,6 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
       } else {  // KL_EPI_QKV_ROPE
         const int region = (int)(n / D);
         const int64_t cc = n - (int64_t)region * D;
-        const int head = (int)(cc >> 7);
         if (region < 2) {
           // the table is pair-major ([64, M] of (c, s)): the 32 lanes (32
           // consecutive rows) read 256 contiguous bytes per pair

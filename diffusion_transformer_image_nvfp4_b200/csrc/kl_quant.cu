@@ -63,23 +63,40 @@ __device__ __forceinline__ GsParams gs_given(float gs) {
   return p;
 }
 
+// 1/S for every scale byte sb (S = e4m3(sb) * gs; 0 when S is 0), computed
+// once per CTA: the same IEEE fp32 multiply and division the encoder would
+// otherwise do per 16-element block, so the codes are unchanged.  sb never
+// exceeds 0x7E (448) after the satfinite conversion.
+__device__ __forceinline__ void fill_rcp_table(float* tab, const GsParams& g) {
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    const float S = __fmul_rn(e4m3_to_f32((uint32_t)i), g.gs);
+    tab[i] = S == 0.f ? 0.f : __fdiv_rn(1.0f, S);
+  }
+}
+
+// y = v * r for eight floats (packed fp32x2 multiplies, RNE) -> eight e2m1
+__device__ __forceinline__ uint32_t scale_to_e2m1x8(const float* v, float r) {
+  const uint64_t r2 = pack_f32x2(r, r);
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) unpack_f32x2(mul_f32x2(pack_f32x2(v[i], v[i + 1]), r2), y[i], y[i + 1]);
+  return f32x8_to_e2m1x8(y);
+}
+
 // Encode 16 values: returns the scale byte, writes 8 packed code bytes.
-__device__ __forceinline__ uint32_t encode_block16(const float (&v)[16], const GsParams& g, uint2& packed) {
+__device__ __forceinline__ uint32_t encode_block16(const float (&v)[16], const GsParams& g, const float* rtab,
+                                                   uint2& packed) {
   float amax_b = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-  uint32_t sb = amax_b > 0.f ? f32_to_e4m3(__fmul_rn(amax_b, g.inv)) : 0u;
-  const float S = __fmul_rn(e4m3_to_f32(sb), g.gs);
-  if (S == 0.f) {
+  const uint32_t sb = amax_b > 0.f ? f32_to_e4m3(__fmul_rn(amax_b, g.inv)) : 0u;
+  const float r = rtab[sb];
+  if (r == 0.f) {
     packed = make_uint2(0u, 0u);
     return sb;
   }
-  const float r = __fdiv_rn(1.0f, S);
-  float y[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(v[i], r);
-  packed.x = f32x8_to_e2m1x8(y);
-  packed.y = f32x8_to_e2m1x8(y + 8);
+  packed.x = scale_to_e2m1x8(v, r);
+  packed.y = scale_to_e2m1x8(v + 8, r);
   return sb;
 }
 
@@ -113,6 +130,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
                                                        int mode) {
   const bool mma = mode & 1, given = mode & 2, perm = mode & 4;
   const GsParams g = given ? gs_given(*gs_io) : gs_from_amax(*amax);
+  __shared__ float rtab[128];
+  fill_rcp_table(rtab, g);
+  __syncthreads();
   const int64_t kbn = cols >> 4;
   const int64_t total = rows_padded * kbn;
   if (!given && blockIdx.x == 0 && threadIdx.x == 0) *gs_io = g.gs;
@@ -127,7 +147,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
     float v[16];
     load16_bf16(x + src * cols + (kb << 4), v);
     uint2 pk;
-    const uint32_t sb = encode_block16(v, g, pk);
+    const uint32_t sb = encode_block16(v, g, rtab, pk);
     *reinterpret_cast<uint2*>(codes + row * (cols >> 1) + (kb << 3)) = pk;
     scales[soff] = (uint8_t)sb;
   }
@@ -203,6 +223,9 @@ __global__ void __launch_bounds__(256) ln_quant_kernel(const uint16_t* __restric
                                                        uint8_t* __restrict__ scales, float* __restrict__ gs_out,
                                                        uint16_t* __restrict__ m_out) {
   const GsParams g = gs_from_amax(*amax);
+  __shared__ float rtab[128];
+  fill_rcp_table(rtab, g);
+  __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = g.gs;
   const int64_t kbn = cols >> 4;
   const int64_t total = rows_padded * kbn;
@@ -229,10 +252,30 @@ __global__ void __launch_bounds__(256) ln_quant_kernel(const uint16_t* __restric
       dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
     uint2 pk;
-    const uint32_t sb = encode_block16(v, g, pk);
+    const uint32_t sb = encode_block16(v, g, rtab, pk);
     *reinterpret_cast<uint2*>(codes + row * (cols >> 1) + (kb << 3)) = pk;
     scales[soff] = (uint8_t)sb;
   }
+}
+
+// m of the 8 elements of one 16-byte chunk (4 words of bf16 pairs each for
+// x, shift, scale): packed fp32x2 RNE steps, the same operations as
+// ln_mod_value (x - mean, * rstd, fma with 1 + scale and shift), then one
+// bf16x2 conversion per pair.  Returns the 4 words of bf16 m.
+__device__ __forceinline__ uint4 ln_mod_chunk(const uint4& xv, const uint4& sh, const uint4& sc, uint64_t negmean2,
+                                              uint64_t rstd2) {
+  const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w}, a[4] = {sh.x, sh.y, sh.z, sh.w}, b[4] = {sc.x, sc.y, sc.z, sc.w};
+  const uint64_t one2 = pack_f32x2(1.0f, 1.0f);
+  uint32_t m[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint64_t y = mul_f32x2(add_f32x2(bf16x2_to_f32x2(w[j]), negmean2), rstd2);
+    const uint64_t onep = add_f32x2(one2, bf16x2_to_f32x2(b[j]));
+    float lo, hi;
+    unpack_f32x2(fma_f32x2(y, onep, bf16x2_to_f32x2(a[j])), lo, hi);
+    m[j] = pack_bf16x2(lo, hi);
+  }
+  return make_uint4(m[0], m[1], m[2], m[3]);
 }
 
 // ------------------------- LayerNorm + modulate, warp per row, NCH chunks
@@ -248,51 +291,51 @@ __global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* _
   constexpr int64_t cols = NCH * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  float lmax = 0.f;
+  uint32_t amax_w = 0u;
   if (row < rows) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
     uint4 xv[NCH];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) xv[c] = __ldg(xr + c * 32 + lane);
-    float s = 0.f;
+    // sums in two packed fp32 chains per lane (a fixed order, so the same
+    // row always gives the same statistics)
+    uint64_t s2[2] = {0ull, 0ull};
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) s += bf16_bits_to_f32(w[j] & 0xFFFFu) + bf16_bits_to_f32(w[j] >> 16);
+      for (int j = 0; j < 4; ++j) s2[j & 1] = add_f32x2(s2[j & 1], bf16x2_to_f32x2(w[j]));
     }
-    const float mean = __fdiv_rn(warp_sum(s), (float)cols);
-    float ss = 0.f;
+    float s0, s1, s2a, s3;
+    unpack_f32x2(s2[0], s0, s1);
+    unpack_f32x2(s2[1], s2a, s3);
+    const float mean = __fdiv_rn(warp_sum((s0 + s1) + (s2a + s3)), (float)cols);
+    const uint64_t negmean2 = pack_f32x2(-mean, -mean);
+    uint64_t q2[2] = {0ull, 0ull};
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float a = bf16_bits_to_f32(w[j] & 0xFFFFu) - mean, b = bf16_bits_to_f32(w[j] >> 16) - mean;
-        ss += a * a + b * b;
+        const uint64_t d = add_f32x2(bf16x2_to_f32x2(w[j]), negmean2);
+        q2[j & 1] = fma_f32x2(d, d, q2[j & 1]);
       }
     }
-    const float rstd = __frsqrt_rn(__fadd_rn(__fdiv_rn(warp_sum(ss), (float)cols), 1e-6f));
+    unpack_f32x2(q2[0], s0, s1);
+    unpack_f32x2(q2[1], s2a, s3);
+    const float rstd = __frsqrt_rn(__fadd_rn(__fdiv_rn(warp_sum((s0 + s1) + (s2a + s3)), (float)cols), 1e-6f));
     if (lane == 0) stats[row] = make_float2(mean, rstd);
+    const uint64_t rstd2 = pack_f32x2(rstd, rstd);
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const uint4 sh = __ldg(reinterpret_cast<const uint4*>(shift) + c * 32 + lane);
       const uint4 sc = __ldg(reinterpret_cast<const uint4*>(scale) + c * 32 + lane);
-      const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-      const uint32_t a[4] = {sh.x, sh.y, sh.z, sh.w}, b[4] = {sc.x, sc.y, sc.z, sc.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t sft = hh ? 16 : 0;
-          const float onep = __fadd_rn(1.0f, bf16_bits_to_f32((b[j] >> sft) & 0xFFFFu));
-          const float mv = ln_mod_value(bf16_bits_to_f32((w[j] >> sft) & 0xFFFFu), mean, rstd, onep,
-                                        bf16_bits_to_f32((a[j] >> sft) & 0xFFFFu));
-          lmax = fmaxf(lmax, fabsf(mv));
-        }
+      const uint4 m = ln_mod_chunk(xv[c], sh, sc, negmean2, rstd2);
+      amax_w = bf16x2_absmax(bf16x2_absmax(amax_w, m.x), m.y);
+      amax_w = bf16x2_absmax(bf16x2_absmax(amax_w, m.z), m.w);
     }
   }
-  lmax = warp_max(lmax);
+  const float lmax = warp_max(bf16x2_hmax_f32(amax_w));
   if (lane == 0 && row < rows) atomic_max_nonneg(amax, lmax);
 }
 
@@ -310,6 +353,9 @@ __global__ void __launch_bounds__(256) ln_quant_rows_kernel(const uint16_t* __re
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
   const GsParams g = gs_from_amax(*amax);
+  __shared__ float rtab[128];
+  fill_rcp_table(rtab, g);
+  __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x == 0) *gs_out = g.gs;
   if (row >= rows_padded) return;
   if (row >= rows) {  // padding rows of the MMA scale layout
@@ -321,41 +367,34 @@ __global__ void __launch_bounds__(256) ln_quant_rows_kernel(const uint16_t* __re
 #pragma unroll
   for (int c = 0; c < NCH; ++c) xv[c] = __ldg(xr + c * 32 + lane);
   const float2 st = stats[row];
+  const uint64_t negmean2 = pack_f32x2(-st.x, -st.x), rstd2 = pack_f32x2(st.y, st.y);
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
     const int64_t col = ((int64_t)c * 32 + lane) * 8;
     const uint4 sh = __ldg(reinterpret_cast<const uint4*>(shift) + c * 32 + lane);
     const uint4 sc = __ldg(reinterpret_cast<const uint4*>(scale) + c * 32 + lane);
-    const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-    const uint32_t a[4] = {sh.x, sh.y, sh.z, sh.w}, b[4] = {sc.x, sc.y, sc.z, sc.w};
-    float v[8];
-    float a8 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t sft = hh ? 16 : 0;
-        const float onep = __fadd_rn(1.0f, bf16_bits_to_f32((b[j] >> sft) & 0xFFFFu));
-        v[2 * j + hh] = ln_mod_value(bf16_bits_to_f32((w[j] >> sft) & 0xFFFFu), st.x, st.y, onep,
-                                     bf16_bits_to_f32((a[j] >> sft) & 0xFFFFu));
-        a8 = fmaxf(a8, fabsf(v[2 * j + hh]));
-      }
-    if (m_out)
-      *reinterpret_cast<uint4*>(m_out + row * cols + col) =
-          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    const uint4 m = ln_mod_chunk(xv[c], sh, sc, negmean2, rstd2);
+    if (m_out) *reinterpret_cast<uint4*>(m_out + row * cols + col) = m;
+    // 16-element block = this lane's 8 values and its neighbour's
+    const float a8 = bf16x2_hmax_f32(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(0u, m.x), m.y), m.z), m.w));
     const float amax_b = fmaxf(a8, __shfl_xor_sync(0xffffffffu, a8, 1));
     const uint32_t sb = amax_b > 0.f ? f32_to_e4m3(__fmul_rn(amax_b, g.inv)) : 0u;
-    const float S = __fmul_rn(e4m3_to_f32(sb), g.gs);
+    const float rr = rtab[sb];
     uint32_t code = 0u;
-    if (S != 0.f) {
-      const float rr = __fdiv_rn(1.0f, S);
-      float y[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], rr);
-      code = f32x8_to_e2m1x8(y);
+    if (rr != 0.f) {
+      const float v[8] = {bf16lo_f32(m.x), bf16hi_f32(m.x), bf16lo_f32(m.y), bf16hi_f32(m.y),
+                          bf16lo_f32(m.z), bf16hi_f32(m.z), bf16lo_f32(m.w), bf16hi_f32(m.w)};
+      code = scale_to_e2m1x8(v, rr);
     }
     *reinterpret_cast<uint32_t*>(codes + row * (cols >> 1) + (col >> 1)) = code;
-    if ((lane & 1) == 0) scales[mma_scale_offset(row, col >> 4, cols)] = (uint8_t)sb;
+    // the chunk's 16 scale bytes (lanes 0, 2, .., 30) are 4 words of the MMA
+    // layout: scale kb = c*16 + lane/2 sits at byte (kb & 3) of its word
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sb, 2);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 4);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sb, 6);
+    if ((lane & 7) == 0)
+      *reinterpret_cast<uint32_t*>(scales + mma_scale_offset(row, col >> 4, cols)) =
+          sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
   }
 }
 
@@ -377,6 +416,7 @@ static cudaError_t launch_ln_rows(const void* x, int64_t rows, const void* shift
 }
 
 // ------------------------------------------------------------ FP8 cast
+constexpr int kFp8MaxHeads = 512;  // ncols / 128 (the launcher checks)
 // 16 elements per thread (inside one 128-wide head).
 __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t ncols,
                                                        int64_t ld, const float* __restrict__ amax,
@@ -384,14 +424,22 @@ __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restric
   const int64_t n16 = ncols >> 4;
   const int64_t total = T * n16;
   const int64_t nheads = ncols >> 7;
-  if (blockIdx.x == 0 && threadIdx.x < nheads) {
-    const float a = amax[threadIdx.x];
-    scales_out[threadIdx.x] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
+  if (blockIdx.x == 0) {
+    for (int hh = threadIdx.x; hh < nheads; hh += blockDim.x) {
+      const float a = amax[hh];
+      scales_out[hh] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
+    }
   }
+  // 448/amax per head (the same IEEE division, once per CTA and head)
+  __shared__ float inv_tab[kFp8MaxHeads];
+  for (int hh = threadIdx.x; hh < nheads; hh += blockDim.x) {
+    const float a = amax[hh];
+    inv_tab[hh] = a > 0.f ? __fdiv_rn(448.0f, a) : 1.0f;
+  }
+  __syncthreads();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / n16, c = (i - t * n16) << 4;
-    const float a = __ldg(amax + (c >> 7));
-    const float inv = a > 0.f ? __fdiv_rn(448.0f, a) : 1.0f;
+    const float inv = inv_tab[c >> 7];
     float v[16];
     load16_bf16(x + t * ld + c, v);
     uint32_t w[4];
@@ -485,6 +533,7 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
 
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s) {
+  if (ncols / 128 > kFp8MaxHeads) return cudaErrorInvalidValue;
   fp8_cast_kernel<<<grid_for(T * (ncols / 16), 256), 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), T, ncols,
                                                                   ld, amax, reinterpret_cast<uint8_t*>(out),
                                                                   scales_out);
