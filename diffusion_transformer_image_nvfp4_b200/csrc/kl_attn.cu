@@ -67,7 +67,8 @@ struct AttnCfg {
   static constexpr int BAR_OFF = P_OFF + QT * 2 * TILE;
   static constexpr int L_OFF = BAR_OFF + 512;      // partial row sums, QT x SPLIT x 128 fp32
   static constexpr int SOFTMAX_THREADS = QT * 128 * SPLIT;
-  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
+  static constexpr int PV_WARP = 2 + SOFTMAX_THREADS / 32;  // after the softmax warps
+  static constexpr int THREADS = 64 + SOFTMAX_THREADS + 32;
   static constexpr uint32_t TMEM_COLS = QT * 256;
   static constexpr int SMEM_BYTES = L_OFF + QT * SPLIT * 128 * 4 + 1024;
   static_assert(SMEM_BYTES <= 232448, "smem budget");
@@ -139,8 +140,8 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   uint64_t* p_empty = p_full + 2 * QT;        // QT x 2
   uint64_t* o_done = p_empty + 2 * QT;        // QT: one phase per P.V
   uint64_t* o_last = o_done + QT;             // QT: the last P.V only
-  uint64_t* drain = o_last + QT;              // 1
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = o_last + QT;              // 2: S issuer, P.V issuer
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);  // K read by the S issuer, V by the P.V issuer
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&s_full[t], 1);
@@ -162,7 +163,8 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
         mbar_init(&p_empty[2 * t + b], 1);
       }
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -217,11 +219,16 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA
-    // The whole warp runs the loop and one elected lane issues; smem
-    // descriptors are built once and advanced by adding offsets (16-byte
-    // units) to the start-address field.
+  } else if (warp == 1 || warp == C::PV_WARP) {
+    // ------------------------------------------------------- MMA issuers
+    // Two warps issue to the tensor core: warp 1 the scores S_t(j) = Q_t K_j^T
+    // (waiting only for K_j and for the softmax to have read S_t(j-1)), the
+    // P.V warp O_t += P_t(j) V_j (waiting for P_t(j)).  The scores of the
+    // next key tile therefore never queue behind a P.V that waits for the
+    // softmax.  Each warp commits its own barriers; a K/V stage is released
+    // by one arrival from each.  One elected lane issues; smem descriptors are
+    // built once and advanced by offsets (16-byte units).
+    const bool s_issuer = warp == 1;
     constexpr uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, 0) : idesc_bf16(128, 128, 0);
     constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, 128, 1) : idesc_bf16(128, 128, 1);
     constexpr uint64_t TILE16 = (uint64_t)(C::TILE >> 4);
@@ -229,20 +236,15 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     const uint64_t k_desc0 = smem_desc(smem_u32(kv_smem), 16, 1024, kLayoutSw128);
     const uint64_t v_desc0 = smem_desc(smem_u32(kv_smem + C::TILE), 16384, 1024, kLayoutSw128);
     const uint64_t p_desc0 = smem_desc(smem_u32(p_smem), 16, 1024, kLayoutSw128);
-    bool ok = warp_wait(q_full, 0, abort_flag);
-    // Issue order per key tile j: for each query tile t, S_t(j) = Q_t K_j^T
-    // then O_t += P_t(j-1) V_{j-1}.
-    for (int j = 0; ok && j <= n; ++j) {
-      const int s = j % C::NS;
-      if (j < n && !warp_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag)) {
+    bool ok = !s_issuer || warp_wait(q_full, 0, abort_flag);
+    for (int j = 0; ok && j < n; ++j) {
+      const int s = j % C::NS, b = j & 1;
+      if (!warp_wait(&kv_full[s], (uint32_t)(j / C::NS) & 1u, abort_flag)) {
         ok = false;
         break;
       }
-      const int jj = j - 1, sp = (jj + C::NS) % C::NS, b = jj & 1;
-      const uint64_t k_desc = k_desc0 + (uint64_t)(2 * s) * TILE16;
-      const uint64_t v_desc = v_desc0 + (uint64_t)(2 * sp) * TILE16;
       for (int t = 0; t < QT && ok; ++t) {
-        if (j < n) {
+        if (s_issuer) {
           if (!warp_wait(&s_empty[t], ((uint32_t)j & 1u) ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -250,6 +252,7 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
           tc_fence_after();
           if (elect_one()) {
             const uint64_t q_desc = q_desc0 + (uint64_t)t * TILE16;
+            const uint64_t k_desc = k_desc0 + (uint64_t)(2 * s) * TILE16;
 #pragma unroll
             for (int kk = 0; kk < C::KSTEPS; ++kk) {
               // K-major step kk: FP8 32 bytes, BF16 16 elements (64-element halves 16 KB apart)
@@ -262,43 +265,43 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
             tc_commit(&s_full[t]);
           }
           __syncwarp();
-        }
-        if (j >= 1) {
-          if (!warp_wait(&p_full[2 * t + b], (uint32_t)(jj >> 1) & 1u, abort_flag)) {
+        } else {
+          if (!warp_wait(&p_full[2 * t + b], (uint32_t)(j >> 1) & 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           if (elect_one()) {
             const uint64_t p_desc = p_desc0 + (uint64_t)(2 * t + b) * TILE16;
+            const uint64_t v_desc = v_desc0 + (uint64_t)(2 * s) * TILE16;
 #pragma unroll
             for (int kk = 0; kk < C::KSTEPS; ++kk) {
               const uint64_t off = FP8 ? (uint64_t)(kk * 2) : (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
               // MN-major V: step kk covers keys [kk*R, kk*R + R), R = 32 (FP8) / 16 (BF16) rows of 128 B
               const uint64_t voff = (uint64_t)(kk * (FP8 ? 32 : 16) * 8);
               if (FP8)
-                mma_f8(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (jj | kk) != 0);
+                mma_f8(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (j | kk) != 0);
               else
-                mma_f16(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (jj | kk) != 0);
+                mma_f16(tmem + t * 256 + 128, p_desc + off, v_desc + voff, id_pv, (j | kk) != 0);
             }
             tc_commit(&o_done[t]);
             tc_commit(&p_empty[2 * t + b]);
-            if (jj == n - 1) tc_commit(&o_last[t]);
+            if (j == n - 1) tc_commit(&o_last[t]);
           }
           __syncwarp();
         }
       }
       if (!ok) break;
-      // K/V stage of tile j-1 is free once the last P.V that reads it is done
-      if (j >= 1) {
-        if (elect_one()) tc_commit(&kv_empty[sp]);
-        __syncwarp();
-      }
+      // this warp's reads of stage s (K or V of tile j) are done once its
+      // MMAs so far have completed
+      if (elect_one()) tc_commit(&kv_empty[s]);
+      __syncwarp();
     }
-    if (elect_one()) tc_commit(drain);
+    uint64_t* my_drain = &drain[s_issuer ? 0 : 1];
+    if (elect_one()) tc_commit(my_drain);
     __syncwarp();
     volatile int no_abort = 0;
-    warp_wait(drain, 0, &no_abort);
+    warp_wait(my_drain, 0, &no_abort);
   } else {
     // ------------------------------------------------------------ softmax
     constexpr int COLS = C::COLS;
