@@ -237,10 +237,10 @@ def gemm_nvfp4_fused(A, W, epilogue="none", out=None, out_dtype=torch.bfloat16, 
 
 
 def rope_table(n_text, grid_h, grid_w, n_ref=0, theta=10000.0, device="cuda"):
-    """kl_rope_table: fp32 (cos, sin) [64, T, 2] (pair-major) for the joint sequence."""
+    """kl_rope_table: fp32 (cos, sin) [16, T, 4, 2] (groups of 4 pairs) for the joint sequence."""
     lay = _TokenLayout(n_text, grid_h, grid_w, n_ref)
     T = lib().kl_layout_tokens(ctypes.byref(lay))
-    cs = torch.empty((64, T, 2), dtype=torch.float32, device=device)
+    cs = torch.empty((16, T, 4, 2), dtype=torch.float32, device=device)
     _check(lib().kl_rope_table(ctypes.byref(lay), theta, cs.data_ptr(), _stream()), "kl_rope_table")
     return cs
 

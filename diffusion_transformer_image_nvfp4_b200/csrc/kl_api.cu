@@ -220,7 +220,7 @@ kl_status kl_gemm_nvfp4_fused(const kl_nvfp4_tensor* A, const kl_nvfp4_tensor* W
     case KL_EPI_QKV_ROPE:
       if (!epi->rope_cs || !epi->amax_out) return KL_ERR_INVALID_ARG;
       if (N % 384 || N / 3 / 128 > 64) return KL_ERR_UNSUPPORTED_SHAPE;
-      if (!aligned(epi->rope_cs, 16)) return KL_ERR_MISALIGNED;
+      if (!aligned(epi->rope_cs, 32)) return KL_ERR_MISALIGNED;  // 32-byte table loads
       break;
     case KL_EPI_SWIGLU:
       if (!epi->amax_out) return KL_ERR_INVALID_ARG;
@@ -379,7 +379,7 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   const kl_nvfp4_tensor* ops[4] = {&w->wqkv, &w->wo, &w->w1, &w->w2};
   for (auto* t : ops)
     if ((st = check_operand(t)) != KL_OK) return st;
-  if (!aligned(io->x, 16) || !aligned(io->out, 16) || !aligned(io->rope_cs, 16)) return KL_ERR_MISALIGNED;
+  if (!aligned(io->x, 16) || !aligned(io->out, 16) || !aligned(io->rope_cs, 32)) return KL_ERR_MISALIGNED;
   const size_t need = kl_block_workspace_size(T, D, H, F, io->attn_precision);
   if (!workspace || ws_bytes < need) return KL_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return KL_ERR_MISALIGNED;

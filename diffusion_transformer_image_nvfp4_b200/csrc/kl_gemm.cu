@@ -196,16 +196,25 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
         const int region = (int)(n / D);
         const int64_t cc = n - (int64_t)region * D;
         if (region < 2) {
-          // the table is pair-major ([64, M] of (c, s)): the 32 lanes (32
-          // consecutive rows) read 256 contiguous bytes per pair
-          const int j0 = (int)((cc & 127) >> 1);
-          const float2* cs = p.rope_cs + (int64_t)j0 * p.M + (valid ? row : 0);
+          // the table holds groups of 4 pairs per token ([16][M][4] of (c, s)):
+          // one 32-byte load gives a thread its row's 4 pairs, and the 32 lanes
+          // (32 consecutive rows) read 1 KB contiguous per load
+          const int j0 = (int)((cc & 127) >> 1);  // multiple of 16
+          const float* cs = reinterpret_cast<const float*>(p.rope_cs) + ((int64_t)(j0 >> 2) * p.M + (valid ? row : 0)) * 8;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float2 t = __ldg(cs + (int64_t)q * p.M);  // (c, s) of pair j0 + q
-            const float a0 = w[2 * q], b0 = w[2 * q + 1];
-            w[2 * q] = a0 * t.x - b0 * t.y;
-            w[2 * q + 1] = a0 * t.y + b0 * t.x;
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float t[8];
+            asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=f"(t[0]), "=f"(t[1]), "=f"(t[2]), "=f"(t[3]), "=f"(t[4]), "=f"(t[5]), "=f"(t[6]),
+                           "=f"(t[7])
+                         : "l"(cs + (int64_t)g4 * p.M * 8));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {  // pair j0 + 4*g4 + u
+              const int q = 4 * g4 + u;
+              const float a0 = w[2 * q], b0 = w[2 * q + 1];
+              w[2 * q] = a0 * t[2 * u] - b0 * t[2 * u + 1];
+              w[2 * q + 1] = a0 * t[2 * u + 1] + b0 * t[2 * u];
+            }
           }
         }
         qkv_amax = fmaxf(qkv_amax, round_bf16x32(*reinterpret_cast<float(*)[32]>(w)));

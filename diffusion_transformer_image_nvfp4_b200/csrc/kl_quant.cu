@@ -454,12 +454,15 @@ __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restric
 // ------------------------------------------------------------ RoPE table
 __global__ void rope_table_kernel(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta,
                                   float2* __restrict__ cs) {
-  // pair-major: cs[j * T + t]
+  // grouped pair-major: the (c, s) of pair j of token t at
+  // cs[(j/4 * T + t) * 4 + j%4]; thread i = (j/4 * T + t) * 4 + j%4
   const int64_t T = n_text + (1 + n_ref) * gh * gw;
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= T * 64) return;
-  const int j = (int)(i / T);
-  const int64_t t = i - (int64_t)j * T;
+  const int64_t gt = i >> 2;
+  const int g = (int)(gt / T);
+  const int64_t t = gt - (int64_t)g * T;
+  const int j = g * 4 + (int)(i & 3);
   double phi;
   if (t < n_text) {
     phi = (double)t * pow(theta, -2.0 * j / 128.0);

@@ -181,7 +181,7 @@ typedef struct kl_epilogue {
   int kind;               /* KL_EPI_* */
   int out_dtype;          /* KL_OUT_BF16 (all kinds) or KL_OUT_F32 (KL_EPI_NONE only) */
   void* out;              /* NONE/GATED_RESIDUAL/QKV_ROPE: [M, N]; SWIGLU: [M, N/2]; row-major */
-  const float* rope_cs;   /* QKV_ROPE: fp32 [64, M, 2] (cos, sin), pair-major (kl_rope_table) */
+  const float* rope_cs;   /* QKV_ROPE: fp32 (cos, sin) table in the kl_rope_table layout, M tokens, 32-byte aligned */
   const void* gate;       /* GATED_RESIDUAL: bf16 [N] */
   const void* residual;   /* GATED_RESIDUAL: bf16 [M, N] (may alias nothing else written) */
   float* amax_out;        /* QKV_ROPE: [3*N/384] per (q|k|v, head) max|out|; SWIGLU: [1].
@@ -208,7 +208,7 @@ typedef struct kl_epilogue {
  *  QKV_ROPE       N = 3*D, D = 128*H.  Columns [0,D) are q, [D,2D) k, [2D,3D)
  *                 v; head h = columns [128h, 128h+128) of each.  q and k pairs
  *                 (2j, 2j+1) are rotated (a,b) -> (a c - b s, a s + b c) with
- *                 (c, s) = rope_cs[j, m]; out is bf16 [M, 3D]; amax_out[r*H+h]
+ *                 (c, s) = rope_cs[j/4, m, j%4]; out is bf16 [M, 3D]; amax_out[r*H+h]
  *                 receives the max |bf16 value| of region r (q,k,v), head h.
  *  SWIGLU         W holds 2F rows in the KL_ROWS_SWIGLU_INTERLEAVE order (each
  *                 128-row group: 64 gate rows then the matching 64 up rows);
@@ -224,8 +224,10 @@ kl_status kl_gemm_nvfp4_fused(const kl_nvfp4_tensor* A, const kl_nvfp4_tensor* W
                               void* stream);
 
 /*
- * kl_rope_table -- fp32 (cos, sin) table [64, T, 2] (pair-major: entry
- * (j, t) at cs_out[2*(j*T + t)]) for the joint sequence
+ * kl_rope_table -- fp32 (cos, sin) table [16, T, 4, 2] (groups of 4 pairs,
+ * token within group: pair j of token t at cs_out[2*((j/4*T + t)*4 + j%4)];
+ * 32-byte aligned rows of 4 pairs, so a consumer thread holding one token
+ * reads 4 pairs with one 32-byte load) for the joint sequence
  * [text (n_text); noisy image (grid_h x grid_w, row-major); n_ref references
  * on grids of the same size].  Reading (RoPE theta 10000 on head dim 128,
  * interleaved pairs): text token i turns pair j by i*theta^(-2j/128); an
@@ -293,7 +295,7 @@ typedef struct kl_block_weights {
 typedef struct kl_block_io {
   const void* x;        /* bf16 [T, D] input residual stream                       */
   const void* mod[6];   /* bf16 [D] each: shift1, scale1, gate1, shift2, scale2, gate2 */
-  const float* rope_cs; /* fp32 [64, T, 2] from kl_rope_table                       */
+  const float* rope_cs; /* fp32 [16, T, 4, 2] from kl_rope_table                    */
   int64_t T, D, H, F;
   int attn_precision;   /* KL_ATTN_FP8 or KL_ATTN_BF16                             */
   void* out;            /* bf16 [T, D] block output (must not alias x)             */

@@ -53,7 +53,8 @@ def test_ln_constant_rows_and_scale_minus_one():
 
 @pytest.mark.parametrize("lay", [(64, 16, 16, 0), (512, 64, 64, 1), (7, 3, 5, 2)])
 def test_rope_table(lay):
-    cs = to_np(kl.rope_table(*lay)).transpose(1, 0, 2)  # pair-major [64, T, 2] -> [T, 64, 2]
+    cs16 = to_np(kl.rope_table(*lay))  # [16, T, 4, 2]: groups of 4 pairs
+    cs = cs16.transpose(1, 0, 2, 3).reshape(cs16.shape[1], 64, 2)
     phi = block.rope_angles(block.TokenLayout(*lay))
     np.testing.assert_allclose(cs[..., 0], np.cos(phi), rtol=0, atol=2e-7)
     np.testing.assert_allclose(cs[..., 1], np.sin(phi), rtol=0, atol=2e-7)
