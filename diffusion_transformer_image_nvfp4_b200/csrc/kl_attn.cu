@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // no global memory before the previous kernel of the stream is done
+  pdl_trigger();
   uint8_t* q_smem = smem + C::Q_OFF;
   uint8_t* kv_smem = smem + C::KV_OFF;
   uint8_t* p_smem = smem + C::P_OFF;
@@ -520,8 +522,7 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int qblocks = (int)((a.T + 128 * C::QT - 1) / (128 * C::QT));
   dim3 grid((unsigned)qblocks, (unsigned)a.H);
-  attn_kernel<FP8><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<FP8>, grid, dim3(C::THREADS), C::SMEM_BYTES, s, tq, tk, tv, p);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {

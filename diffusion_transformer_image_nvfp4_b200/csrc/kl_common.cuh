@@ -101,6 +101,17 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation, so it may start while the previous
+// kernel of the stream is finishing: it does its setup (barriers, TMEM,
+// tensor-map prefetch), then pdl_wait() -- which returns once the previous
+// grid has completed and its memory is visible -- before touching any global
+// memory.  pdl_trigger() lets the next kernel launch once every CTA of this
+// grid has started (so waiting dependents never hold SM resources that this
+// grid's remaining CTAs need).  Without a preceding launch both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------- TMA and bulk
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {

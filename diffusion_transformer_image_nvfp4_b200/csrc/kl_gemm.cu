@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(352, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // no global memory before the previous kernel of the stream is done
+  pdl_trigger();
 
   // Shared-memory descriptors of stage 0; a stage or K-step offset is added
   // in 16-byte units to the start-address field (no carry: smem < 256 KB).
@@ -587,6 +589,8 @@ __global__ void __launch_bounds__(352, 1)
   cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // no global memory before the previous kernel of the stream is done
+  pdl_trigger();
   const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
   const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
   const int num_m2 = (int)((p.M + 255) / 256);
@@ -820,13 +824,15 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
   cfg.blockDim = dim3(352);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN>, ta, tb, tsa, tsb, p);
 }
 
@@ -864,8 +870,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  gemm_nvfp4_kernel<BN, KS><<<grid, 352, C::SMEM_BYTES, s>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_nvfp4_kernel<BN, KS>, dim3(grid), dim3(352), C::SMEM_BYTES, s, ta, tb, p);
 }
 
 #ifndef KL_GEMM_KSTEPS

@@ -11,13 +11,32 @@ constexpr int kNumSMs = 148;  // B200; only caps grid-stride grids (persistent k
 
 int device_sm_count();  // cached per process
 
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger
+// in kl_common.cuh); every library kernel waits before its first global access.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // HBM-bound kernels (kl_quant.cu)
 cudaError_t launch_amax_bf16(const void* x, int64_t n, float* amax, cudaStream_t s);
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols, void* codes, void* scales, float* gs_io,
                             const float* amax, int mode, cudaStream_t s);
 cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t cols, const void* shift,
                                         const void* scale, void* codes, void* scales, float* gs_out,
-                                        void* m_out, float2* stats, float* amax, cudaStream_t s);
+                                        void* m_out, float2* stats, float* amax, cudaStream_t s,
+                                        bool amax_zeroed = false);  // true: the caller zeroed amax[0] on s
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s);
 cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,

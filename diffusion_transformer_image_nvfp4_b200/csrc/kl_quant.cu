@@ -21,6 +21,8 @@ constexpr float kGsDivisor = 2688.0f;  // 6 * 448
 // the launcher zeroes first).  Non-finite input sets KL_DEVERR_NONFINITE.
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict__ x, int64_t n8,
                                                         float* __restrict__ amax) {
+  pdl_wait();
+  pdl_trigger();
   float m = 0.f;
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
@@ -128,6 +130,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                        float* __restrict__ gs_io, const float* __restrict__ amax,
                                                        int mode) {
+  pdl_wait();
+  pdl_trigger();
   const bool mma = mode & 1, given = mode & 2, perm = mode & 4;
   const GsParams g = given ? gs_given(*gs_io) : gs_from_amax(*amax);
   __shared__ float rtab[128];
@@ -165,6 +169,8 @@ __global__ void __launch_bounds__(256) ln_stats_amax_kernel(const uint16_t* __re
                                                             int64_t cols, const uint16_t* __restrict__ shift,
                                                             const uint16_t* __restrict__ scale,
                                                             float2* __restrict__ stats, float* __restrict__ amax) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + warp;
   float m = 0.f;
@@ -222,6 +228,8 @@ __global__ void __launch_bounds__(256) ln_quant_kernel(const uint16_t* __restric
                                                        const float* __restrict__ amax, uint8_t* __restrict__ codes,
                                                        uint8_t* __restrict__ scales, float* __restrict__ gs_out,
                                                        uint16_t* __restrict__ m_out) {
+  pdl_wait();
+  pdl_trigger();
   const GsParams g = gs_from_amax(*amax);
   __shared__ float rtab[128];
   fill_rcp_table(rtab, g);
@@ -288,6 +296,8 @@ __global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* _
                                                             const uint16_t* __restrict__ shift,
                                                             const uint16_t* __restrict__ scale,
                                                             float2* __restrict__ stats, float* __restrict__ amax) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int64_t cols = NCH * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
@@ -349,6 +359,8 @@ __global__ void __launch_bounds__(256) ln_quant_rows_kernel(const uint16_t* __re
                                                             const float* __restrict__ amax,
                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                             float* __restrict__ gs_out, uint16_t* __restrict__ m_out) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int64_t cols = NCH * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
@@ -405,14 +417,13 @@ static cudaError_t launch_ln_rows(const void* x, int64_t rows, const void* shift
   const uint16_t* xp = reinterpret_cast<const uint16_t*>(x);
   const uint16_t* shp = reinterpret_cast<const uint16_t*>(shift);
   const uint16_t* scp = reinterpret_cast<const uint16_t*>(scale);
-  ln_stats_rows_kernel<NCH><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(xp, rows, shp, scp, stats, amax);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(ln_stats_rows_kernel<NCH>, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, s, xp, rows,
+                             shp, scp, stats, amax);
   if (e != cudaSuccess) return e;
   const int64_t rows_padded = ((rows + 127) / 128) * 128;
-  ln_quant_rows_kernel<NCH><<<(unsigned)((rows_padded + 7) / 8), 256, 0, s>>>(
-      xp, rows, rows_padded, shp, scp, stats, amax, reinterpret_cast<uint8_t*>(codes),
-      reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
-  return cudaGetLastError();
+  return launch_pdl(ln_quant_rows_kernel<NCH>, dim3((unsigned)((rows_padded + 7) / 8)), dim3(256), 0, s, xp, rows,
+                    rows_padded, shp, scp, stats, (const float*)amax, reinterpret_cast<uint8_t*>(codes),
+                    reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
 }
 
 // ------------------------------------------------------------ FP8 cast
@@ -421,6 +432,8 @@ constexpr int kFp8MaxHeads = 512;  // ncols / 128 (the launcher checks)
 __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t ncols,
                                                        int64_t ld, const float* __restrict__ amax,
                                                        uint8_t* __restrict__ out, float* __restrict__ scales_out) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n16 = ncols >> 4;
   const int64_t total = T * n16;
   const int64_t nheads = ncols >> 7;
@@ -454,6 +467,8 @@ __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restric
 // ------------------------------------------------------------ RoPE table
 __global__ void rope_table_kernel(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta,
                                   float2* __restrict__ cs) {
+  pdl_wait();
+  pdl_trigger();
   // grouped pair-major: the (c, s) of pair j of token t at
   // cs[(j/4 * T + t) * 4 + j%4]; thread i = (j/4 * T + t) * 4 + j%4
   const int64_t T = n_text + (1 + n_ref) * gh * gw;
@@ -490,23 +505,22 @@ static int grid_for(int64_t work, int threads) {
 cudaError_t launch_amax_bf16(const void* x, int64_t n, float* amax, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return e;
-  amax_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), n / 8, amax);
-  return cudaGetLastError();
+  return launch_pdl(amax_bf16_kernel, dim3(grid_for(n / 8, 256)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x),
+                    n / 8, amax);
 }
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols, void* codes, void* scales, float* gs_io,
                             const float* amax, int mode, cudaStream_t s) {
   const int64_t rows_padded = (mode & 1) ? ((rows + 127) / 128) * 128 : rows;
-  quantize_kernel<<<grid_for(rows_padded * (cols / 16), 256), 256, 0, s>>>(
-      reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<uint8_t*>(codes),
-      reinterpret_cast<uint8_t*>(scales), gs_io, amax, mode);
-  return cudaGetLastError();
+  return launch_pdl(quantize_kernel, dim3(grid_for(rows_padded * (cols / 16), 256)), dim3(256), 0, s,
+                    reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<uint8_t*>(codes),
+                    reinterpret_cast<uint8_t*>(scales), gs_io, amax, mode);
 }
 
 cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t cols, const void* shift,
                                         const void* scale, void* codes, void* scales, float* gs_out,
-                                        void* m_out, float2* stats, float* amax, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+                                        void* m_out, float2* stats, float* amax, cudaStream_t s, bool amax_zeroed) {
+  cudaError_t e = amax_zeroed ? cudaSuccess : cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return e;
   if (cols % 256 == 0) {
     switch (cols / 256) {
@@ -521,35 +535,32 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
   }
   // generic widths: row loop per lane, then one thread per 16-element block
   const int64_t blocks = (rows + 7) / 8;
-  ln_stats_amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), rows, cols,
-                                                        reinterpret_cast<const uint16_t*>(shift),
-                                                        reinterpret_cast<const uint16_t*>(scale), stats, amax);
-  e = cudaGetLastError();
+  e = launch_pdl(ln_stats_amax_kernel, dim3((unsigned)blocks), dim3(256), 0, s, reinterpret_cast<const uint16_t*>(x),
+                 rows, cols, reinterpret_cast<const uint16_t*>(shift), reinterpret_cast<const uint16_t*>(scale), stats,
+                 amax);
   if (e != cudaSuccess) return e;
   const int64_t rows_padded = ((rows + 127) / 128) * 128;
-  ln_quant_kernel<<<grid_for(rows_padded * (cols / 16), 256), 256, 0, s>>>(
-      reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<const uint16_t*>(shift),
-      reinterpret_cast<const uint16_t*>(scale), stats, amax, reinterpret_cast<uint8_t*>(codes),
-      reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
-  return cudaGetLastError();
+  return launch_pdl(ln_quant_kernel, dim3(grid_for(rows_padded * (cols / 16), 256)), dim3(256), 0, s,
+                    reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded,
+                    reinterpret_cast<const uint16_t*>(shift), reinterpret_cast<const uint16_t*>(scale),
+                    (const float2*)stats, (const float*)amax, reinterpret_cast<uint8_t*>(codes),
+                    reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
 }
 
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s) {
   if (ncols / 128 > kFp8MaxHeads) return cudaErrorInvalidValue;
-  fp8_cast_kernel<<<grid_for(T * (ncols / 16), 256), 256, 0, s>>>(reinterpret_cast<const uint16_t*>(x), T, ncols,
-                                                                  ld, amax, reinterpret_cast<uint8_t*>(out),
-                                                                  scales_out);
-  return cudaGetLastError();
+  return launch_pdl(fp8_cast_kernel, dim3(grid_for(T * (ncols / 16), 256)), dim3(256), 0, s,
+                    reinterpret_cast<const uint16_t*>(x), T, ncols, ld, amax, reinterpret_cast<uint8_t*>(out),
+                    scales_out);
 }
 
 cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,
                               cudaStream_t s) {
   const int64_t T = n_text + (1 + n_ref) * gh * gw;
   const int64_t n = T * 64;
-  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(n_text, gh, gw, n_ref, theta,
-                                                               reinterpret_cast<float2*>(cs));
-  return cudaGetLastError();
+  return launch_pdl(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, n_text, gh, gw, n_ref,
+                    theta, reinterpret_cast<float2*>(cs));
 }
 
 }  // namespace kl
