@@ -404,8 +404,13 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   };
   mark(0);
   // 1. m1 = bf16(LN(x)(1+scale1)+shift1) -> NVFP4
-  KL_TRY(launch_ln_modulate_quantize(io->x, T, D, io->mod[0], io->mod[1], ws.acodes, ws.ascales, &gs[0], nullptr,
-                                     ws.stats, ln1, s, /*amax_zeroed=*/true));
+  // (m1 goes through the attention-output buffer, free until step 4)
+  if (D % 256 == 0 && D <= 4096)
+    KL_TRY(launch_ln_modulate_quantize_via_m(io->x, T, D, io->mod[0], io->mod[1], ws.acodes, ws.ascales, &gs[0],
+                                             ws.o, ws.stats, ln1, s));
+  else
+    KL_TRY(launch_ln_modulate_quantize(io->x, T, D, io->mod[0], io->mod[1], ws.acodes, ws.ascales, &gs[0], nullptr,
+                                       ws.stats, ln1, s, /*amax_zeroed=*/true));
   mark(1);
   // 2. qkv = m1 Wqkv^T with RoPE on q, k and per-head amax
   GemmArgs g{};
@@ -470,8 +475,13 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   KL_TRY(launch_gemm_nvfp4(g, s));
   mark(6);
   // 7. m2 = bf16(LN(x1)(1+scale2)+shift2) -> NVFP4
-  KL_TRY(launch_ln_modulate_quantize(ws.x1, T, D, io->mod[3], io->mod[4], ws.acodes, ws.ascales, &gs[2], nullptr,
-                                     ws.stats, ln2, s, /*amax_zeroed=*/true));
+  // (m2 goes through the attention-output buffer, free again after step 5)
+  if (D % 256 == 0 && D <= 4096)
+    KL_TRY(launch_ln_modulate_quantize_via_m(ws.x1, T, D, io->mod[3], io->mod[4], ws.acodes, ws.ascales, &gs[2],
+                                             ws.o, ws.stats, ln2, s));
+  else
+    KL_TRY(launch_ln_modulate_quantize(ws.x1, T, D, io->mod[3], io->mod[4], ws.acodes, ws.ascales, &gs[2], nullptr,
+                                       ws.stats, ln2, s, /*amax_zeroed=*/true));
   mark(7);
   // 8. h = bf16(silu(g) u), [g u] = m2 W1^T, + amax
   g = GemmArgs{};

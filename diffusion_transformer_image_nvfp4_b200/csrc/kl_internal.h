@@ -37,6 +37,9 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
                                         const void* scale, void* codes, void* scales, float* gs_out,
                                         void* m_out, float2* stats, float* amax, cudaStream_t s,
                                         bool amax_zeroed = false);  // true: the caller zeroed amax[0] on s
+cudaError_t launch_ln_modulate_quantize_via_m(const void* x, int64_t rows, int64_t cols, const void* shift,
+                                             const void* scale, void* codes, void* scales, float* gs_out,
+                                             void* m_buf, float2* stats, float* amax, cudaStream_t s);
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s);
 cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,

@@ -295,7 +295,8 @@ template <int NCH>
 __global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                             const uint16_t* __restrict__ shift,
                                                             const uint16_t* __restrict__ scale,
-                                                            float2* __restrict__ stats, float* __restrict__ amax) {
+                                                            float2* __restrict__ stats, float* __restrict__ amax,
+                                                            uint16_t* __restrict__ m_out) {
   pdl_wait();
   pdl_trigger();
   constexpr int64_t cols = NCH * 256;
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* _
       const uint4 sh = __ldg(reinterpret_cast<const uint4*>(shift) + c * 32 + lane);
       const uint4 sc = __ldg(reinterpret_cast<const uint4*>(scale) + c * 32 + lane);
       const uint4 m = ln_mod_chunk(xv[c], sh, sc, negmean2, rstd2);
+      if (m_out) reinterpret_cast<uint4*>(m_out + row * cols)[c * 32 + lane] = m;
       amax_w = bf16x2_absmax(bf16x2_absmax(amax_w, m.x), m.y);
       amax_w = bf16x2_absmax(bf16x2_absmax(amax_w, m.z), m.w);
     }
@@ -418,7 +420,7 @@ static cudaError_t launch_ln_rows(const void* x, int64_t rows, const void* shift
   const uint16_t* shp = reinterpret_cast<const uint16_t*>(shift);
   const uint16_t* scp = reinterpret_cast<const uint16_t*>(scale);
   cudaError_t e = launch_pdl(ln_stats_rows_kernel<NCH>, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, s, xp, rows,
-                             shp, scp, stats, amax);
+                             shp, scp, stats, amax, (uint16_t*)nullptr);
   if (e != cudaSuccess) return e;
   const int64_t rows_padded = ((rows + 127) / 128) * 128;
   return launch_pdl(ln_quant_rows_kernel<NCH>, dim3((unsigned)((rows_padded + 7) / 8)), dim3(256), 0, s, xp, rows,
@@ -545,6 +547,35 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
                     reinterpret_cast<const uint16_t*>(shift), reinterpret_cast<const uint16_t*>(scale),
                     (const float2*)stats, (const float*)amax, reinterpret_cast<uint8_t*>(codes),
                     reinterpret_cast<uint8_t*>(scales), gs_out, reinterpret_cast<uint16_t*>(m_out));
+}
+
+// LN + adaLN + NVFP4 as two passes over a materialised m: the statistics
+// pass also stores m (bf16, rows x cols into m_buf), then the standalone
+// quantiser encodes m with gs from the same amax -- the codes the fused
+// encoder would produce (it encodes the same bf16 m), from a kernel with one
+// thread per 16-element block.  Widths cols = 256 * {1, 2, 4, 8, 12, 16};
+// returns cudaErrorInvalidValue for others.  amax[0] must be zero on s.
+cudaError_t launch_ln_modulate_quantize_via_m(const void* x, int64_t rows, int64_t cols, const void* shift,
+                                             const void* scale, void* codes, void* scales, float* gs_out,
+                                             void* m_buf, float2* stats, float* amax, cudaStream_t s) {
+  if (cols % 256) return cudaErrorInvalidValue;
+  const uint16_t* xp = reinterpret_cast<const uint16_t*>(x);
+  const uint16_t* shp = reinterpret_cast<const uint16_t*>(shift);
+  const uint16_t* scp = reinterpret_cast<const uint16_t*>(scale);
+  uint16_t* mp = reinterpret_cast<uint16_t*>(m_buf);
+  const dim3 grid((unsigned)((rows + 7) / 8)), block(256);
+  cudaError_t e;
+  switch (cols / 256) {
+    case 1: e = launch_pdl(ln_stats_rows_kernel<1>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    case 2: e = launch_pdl(ln_stats_rows_kernel<2>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    case 4: e = launch_pdl(ln_stats_rows_kernel<4>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    case 8: e = launch_pdl(ln_stats_rows_kernel<8>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    case 12: e = launch_pdl(ln_stats_rows_kernel<12>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    case 16: e = launch_pdl(ln_stats_rows_kernel<16>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  return launch_quantize(m_buf, rows, cols, codes, scales, gs_out, amax, 1, s);
 }
 
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
