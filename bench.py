@@ -512,6 +512,68 @@ def run_ours(args, wl):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------ DiT loop (c4)
+def run_dit(args):
+    """Per-image latency of the synthetic DiT loop (5 per-mode + 28 joint
+    blocks at the 1024^2 T2I shape, 16 Euler steps), the 16 steps captured in
+    one CUDA graph; weights and inputs drawn on the GPU (seeded)."""
+    import diffusion_transformer_image_nvfp4_b200 as kl
+    from synth import DIT_CONFIGS, dit_inputs
+
+    cfg = DIT_CONFIGS["dit_t2i_1024"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = dit_inputs(cfg, device=dev)
+    blocks = lambda bl: [kl.prepare_block_weights(b["wqkv"], b["wo"], b["w1"], b["w2"]) for b in bl]
+    W = kl.DitWeights(kl.quantize_nvfp4(d["w_in"]), blocks(d["mode_text"]), blocks(d["mode_image"]),
+                      blocks(d["joint"]), kl.quantize_nvfp4(d["w_out"]))
+    for k in ("w_in", "w_out", "mode_text", "mode_image", "joint"):
+        del d[k]
+    torch.cuda.empty_cache()
+    shape = kl.DitShape(cfg.n_text, cfg.grid_h, cfg.grid_w, cfg.channels, cfg.hidden, cfg.heads, cfg.mlp_hidden,
+                        cfg.n_mode, cfg.n_joint, cfg.attn)
+    ropes = (kl.rope_table(cfg.n_text, 0, 0, device=dev), kl.rope_table(0, cfg.grid_h, cfg.grid_w, device=dev),
+             kl.rope_table(cfg.n_text, cfg.grid_h, cfg.grid_w, device=dev))
+    ws = torch.empty(kl.dit_workspace_size(shape), dtype=torch.uint8, device=dev)
+    w_abi = W.abi()
+    ts = [1.0 - i / cfg.n_steps for i in range(cfg.n_steps + 1)]
+    mods = [(d["mod_mode"][i].contiguous(), d["mod_joint"][i].contiguous(), d["mod_final"][i].contiguous())
+            for i in range(cfg.n_steps)]
+    lat0 = d["latent"].contiguous()
+    lat = lat0.clone()
+
+    def image():
+        for i in range(cfg.n_steps):
+            kl.dit_step(shape, W, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i], workspace=ws, w_abi=w_abi)
+
+    image()  # warm-up (eager)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        image()
+    times = []
+    for _ in range(args.warmup + args.steps):
+        lat.copy_(lat0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in times[args.warmup:]]
+    st = kl.device_status()
+    fin = bool(torch.isfinite(lat).all().item())
+    blocks_per_image = cfg.n_steps * (2 * cfg.n_mode + cfg.n_joint)
+    print(json.dumps({"metric": "per-image DiT latency, synthetic 1024^2 T2I loop", "value": round(statistics.median(ms), 3),
+                      "unit": "ms", "higher_is_better": False, "images": args.steps, "warmup": args.warmup,
+                      "config": {"workload": cfg.name, "steps": cfg.n_steps, "per_mode_blocks": cfg.n_mode,
+                                 "joint_blocks": cfg.n_joint, "tokens": cfg.n_text + cfg.grid_h * cfg.grid_w,
+                                 "latent": [2 * cfg.grid_h, 2 * cfg.grid_w, cfg.channels],
+                                 "block_calls_per_image": blocks_per_image,
+                                 "launch": "16 Euler steps captured in one CUDA graph"},
+                      "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,10 +582,14 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="t2i_1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dit", action="store_true", help="time the synthetic DiT loop instead (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
+    if args.dit:
+        run_dit(args)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:

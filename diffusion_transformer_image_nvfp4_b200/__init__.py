@@ -19,6 +19,7 @@ from .build import LIB_PATH
 __all__ = [
     "KLError", "lib", "NVFP4", "quantize_nvfp4", "ln_modulate_quantize_nvfp4", "gemm_nvfp4_fused",
     "rope_table", "cast_fp8_per_head", "joint_attention", "BlockWeights", "prepare_block_weights",
+    "DitShape", "DitWeights", "dit_step", "dit_workspace_size",
     "joint_block_forward", "block_workspace_size", "device_status", "scales_mma_to_linear",
 ]
 
@@ -67,6 +68,24 @@ class _BlockIO(ctypes.Structure):
                 ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
 
 
+class _DitShape(ctypes.Structure):
+    _fields_ = [("n_text", ctypes.c_int64), ("grid_h", ctypes.c_int64), ("grid_w", ctypes.c_int64),
+                ("channels", ctypes.c_int64), ("D", ctypes.c_int64), ("H", ctypes.c_int64), ("F", ctypes.c_int64),
+                ("n_mode_blocks", ctypes.c_int), ("n_joint_blocks", ctypes.c_int), ("attn_precision", ctypes.c_int)]
+
+
+class _DitWeights(ctypes.Structure):
+    _fields_ = [("w_in", _NVFP4Tensor), ("mode_text", ctypes.POINTER(_BlockWeights)),
+                ("mode_image", ctypes.POINTER(_BlockWeights)), ("joint", ctypes.POINTER(_BlockWeights)),
+                ("w_out", _NVFP4Tensor)]
+
+
+class _DitStepIO(ctypes.Structure):
+    _fields_ = [("latent", ctypes.c_void_p), ("text", ctypes.c_void_p), ("mod_mode", ctypes.c_void_p),
+                ("mod_joint", ctypes.c_void_p), ("mod_final", ctypes.c_void_p), ("rope_text", ctypes.c_void_p),
+                ("rope_image", ctypes.c_void_p), ("rope_joint", ctypes.c_void_p), ("dt", ctypes.c_float)]
+
+
 _LIB = None
 _VP, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 _SIGS = {
@@ -88,6 +107,9 @@ _SIGS = {
     "kl_joint_attention_fp8": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _I64, _I64, _I64, _I, _VP, _VP, _VP], _I),
     "kl_block_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
     "kl_joint_block_forward": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
+    "kl_dit_workspace_size": ([ctypes.POINTER(_DitShape)], _SZ),
+    "kl_dit_step": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitWeights), ctypes.POINTER(_DitStepIO), _VP, _SZ,
+                     _VP], _I),
 }
 
 
@@ -320,6 +342,71 @@ def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, wo
     _check(lib().kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(), workspace.numel(),
                                         _stream()), "kl_joint_block_forward")
     return out
+
+
+# ------------------------------------------------------------------ DiT step
+@dataclass
+class DitShape:
+    n_text: int
+    grid_h: int
+    grid_w: int
+    channels: int
+    D: int
+    H: int
+    F: int
+    n_mode_blocks: int
+    n_joint_blocks: int
+    attn: str = "fp8"
+
+    def abi(self):
+        return _DitShape(self.n_text, self.grid_h, self.grid_w, self.channels, self.D, self.H, self.F,
+                         self.n_mode_blocks, self.n_joint_blocks, ATTN[self.attn])
+
+
+@dataclass
+class DitWeights:
+    w_in: NVFP4            # [D, 4*channels]
+    mode_text: list        # [n_mode_blocks] BlockWeights
+    mode_image: list       # [n_mode_blocks] BlockWeights
+    joint: list            # [n_joint_blocks] BlockWeights
+    w_out: NVFP4           # [4*channels, D]
+
+    def abi(self):
+        def arr(blocks):
+            if not blocks:
+                return None
+            return (_BlockWeights * len(blocks))(*[b.abi() for b in blocks])
+        # keep the ctypes arrays alive with the struct
+        self._arrays = (arr(self.mode_text), arr(self.mode_image), arr(self.joint))
+        ptr = lambda a: ctypes.cast(a, ctypes.POINTER(_BlockWeights)) if a is not None else None
+        return _DitWeights(self.w_in.abi(), ptr(self._arrays[0]), ptr(self._arrays[1]), ptr(self._arrays[2]),
+                           self.w_out.abi())
+
+
+def dit_workspace_size(shape):
+    sh = shape.abi()
+    return lib().kl_dit_workspace_size(ctypes.byref(sh))
+
+
+def dit_step(shape, weights, latent, text, mod_mode, mod_joint, mod_final, rope_text, rope_image, rope_joint, dt,
+             workspace=None, w_abi=None):
+    """kl_dit_step: one Euler step, latent (fp32 [2gh, 2gw, C], CUDA) updated in
+    place.  mod_mode bf16 [n_mode, 2, 6, D]; mod_joint bf16 [n_joint, 6, D];
+    mod_final bf16 [2, D]; rope tables from rope_table for the text-only,
+    image-only and joint layouts.  ``w_abi`` (optional): a cached
+    weights.abi() (the ctypes struct), to keep host work out of loops."""
+    _need(latent, torch.float32, "latent")
+    _need(text, torch.bfloat16, "text")
+    sh = shape.abi()
+    need = lib().kl_dit_workspace_size(ctypes.byref(sh))
+    if workspace is None:
+        workspace = _workspace(need, latent.device, "dit")
+    w = weights.abi() if w_abi is None else w_abi
+    io = _DitStepIO(latent.data_ptr(), text.data_ptr(), _ptr(mod_mode), _ptr(mod_joint), mod_final.data_ptr(),
+                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt))
+    _check(lib().kl_dit_step(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
+                             workspace.numel(), _stream()), "kl_dit_step")
+    return latent
 
 
 def device_status(clear=True):

@@ -5,3 +5,4 @@
 #include "kl_attn.cu"
 #include "kl_api.cu"
 #include "kl_noalloc.cu"
+#include "kl_dit.cu"

@@ -337,6 +337,59 @@ size_t kl_block_workspace_size(int64_t T, int64_t D, int64_t H, int64_t F, int a
 kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* io,
                                  void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * kl_dit_step -- one Euler step of a synthetic DiT on the block above ([P2]
+ * Summary: per-mode blocks for each stream, then joint blocks; [P4] The VAE
+ * and Tokenization: 2x2 latent patches; Two-Stage Processing).  Readings
+ * (the pages stop at the block structure):
+ *   patches p[t][k] = bf16(latent[y][x][c]), t = (y/2)*grid_w + x/2,
+ *     k = 4c + 2(y%2) + (x%2)                       (no bias, no norm)
+ *   image tokens = NVFP4(p) . w_in^T (bf16); the text conditioning [n_text, D]
+ *     is copied in front of them each step: sequence [text; image]
+ *   per-mode block i: the block on the text rows alone (mode_text[i], text
+ *     RoPE layout) and on the image rows alone (mode_image[i], image layout)
+ *   joint block i: the block on the whole sequence (joint layout)
+ *   v = NVFP4(bf16(LN(img)*(1+scale_f)+shift_f)) . w_out^T   (fp32 [Ti, 4C])
+ *   latent[y][x][c] = fl(latent + fl(dt * v[t][k]))  (Euler, same (t, k) map)
+ * Shapes: latent fp32 [2*grid_h, 2*grid_w, channels], 4*channels % 128 == 0;
+ * D = 128*H; the block constraints.  mode_text / mode_image / joint are host
+ * arrays (n_mode_blocks / n_joint_blocks entries) of device weights.  Every
+ * pointer in kl_dit_step_io is a device pointer; rope_* come from
+ * kl_rope_table for the layouts (n_text,0,0,0), (0,grid_h,grid_w,0),
+ * (n_text,grid_h,grid_w,0).  workspace >= kl_dit_workspace_size, 256-byte
+ * aligned.  The call is capturable in a CUDA graph (no host sync).
+ */
+typedef struct kl_dit_shape {
+  int64_t n_text, grid_h, grid_w, channels;
+  int64_t D, H, F;
+  int n_mode_blocks, n_joint_blocks;
+  int attn_precision; /* KL_ATTN_FP8 or KL_ATTN_BF16 */
+} kl_dit_shape;
+
+typedef struct kl_dit_weights {
+  kl_nvfp4_tensor w_in;               /* [D, 4*channels] */
+  const kl_block_weights* mode_text;  /* host array [n_mode_blocks] */
+  const kl_block_weights* mode_image; /* host array [n_mode_blocks] */
+  const kl_block_weights* joint;      /* host array [n_joint_blocks] */
+  kl_nvfp4_tensor w_out;              /* [4*channels, D] */
+} kl_dit_weights;
+
+typedef struct kl_dit_step_io {
+  float* latent;           /* fp32 [2*grid_h, 2*grid_w, channels], updated in place */
+  const void* text;        /* bf16 [n_text, D] */
+  const void* mod_mode;    /* bf16 [n_mode_blocks][2 (text, image)][6][D] (block order of kl_block_io.mod) */
+  const void* mod_joint;   /* bf16 [n_joint_blocks][6][D] */
+  const void* mod_final;   /* bf16 [2][D]: shift_f, scale_f */
+  const float* rope_text;
+  const float* rope_image;
+  const float* rope_joint;
+  float dt;                /* t_{i+1} - t_i */
+} kl_dit_step_io;
+
+size_t kl_dit_workspace_size(const kl_dit_shape* shape);
+kl_status kl_dit_step(const kl_dit_shape* shape, const kl_dit_weights* w, const kl_dit_step_io* io,
+                      void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -97,3 +97,76 @@ def uniform_int(shape, low, high, seed):
     """Seeded integers in [low, high) as an int64 tensor."""
     g = torch.Generator().manual_seed(seed)
     return torch.randint(low, high, shape, generator=g, dtype=torch.int64)
+
+
+# ------------------------------------------------------------- DiT loop
+@dataclass(frozen=True)
+class DitConfig:
+    """A synthetic DiT: latent [2*grid_h, 2*grid_w, channels] (2x2 patches ->
+    grid_h x grid_w image tokens of 4*channels features), n_text text tokens,
+    n_mode per-mode blocks then n_joint joint blocks, n_steps Euler steps."""
+
+    name: str
+    n_text: int
+    grid_h: int
+    grid_w: int
+    channels: int
+    hidden: int
+    heads: int
+    mlp_hidden: int
+    n_mode: int
+    n_joint: int
+    n_steps: int
+    attn: str
+    seed: int
+
+
+# c4: a 1024x1024 image -> 128x128x32 latent -> 64x64 tokens of 128 features,
+# 512 text tokens, 5 per-mode + 28 joint blocks, 16 steps; seed 3 (config
+# index - 1).  dit_tiny: the same structure at block-test sizes.
+DIT_CONFIGS = {
+    c.name: c
+    for c in [
+        DitConfig("dit_tiny", 16, 4, 4, 32, 128, 1, 384, 1, 2, 2, "bf16", 11),
+        DitConfig("dit_t2i_1024", 512, 64, 64, 32, 3072, 24, 9216, 5, 28, 16, "fp8", 3),
+    ]
+}
+
+
+def dit_inputs(cfg, with_weights=True, device="cpu"):
+    """Seeded inputs of a DiT run as CPU tensors.  Draw order: latent (fp32
+    N(0,1)); text (bf16 N(0,1)); w_in [D, 4C], w_out [4C, D] (N(0,0.02));
+    per-mode blocks i = 0..n_mode-1: text weights then image weights (each
+    Wqkv, Wo, W1, W2 as in block_inputs); joint blocks; modulation vectors
+    (N(0,0.1)): mode [n_mode, 2, 6, D], joint [n_joint, 6, D], final [2, D]
+    for each of the n_steps steps ([n_steps, ...]).  ``device``: where the
+    generator and tensors live (a CUDA generator draws different numbers than
+    the CPU one; the parity tests use the CPU draws)."""
+    if isinstance(cfg, str):
+        cfg = DIT_CONFIGS[cfg]
+    g = torch.Generator(device=device).manual_seed(cfg.seed)
+    D, F, C = cfg.hidden, cfg.mlp_hidden, cfg.channels
+
+    def _randn(gen, shape, std):
+        return (torch.randn(*shape, generator=gen, dtype=torch.float32, device=device) * std).to(torch.bfloat16)
+
+    out = {"latent": torch.randn(2 * cfg.grid_h, 2 * cfg.grid_w, C, generator=g, dtype=torch.float32,
+                                 device=device),
+           "text": _randn(g, (cfg.n_text, D), 1.0)}
+
+    def block_w():
+        return {"wqkv": _randn(g, (3 * D, D), 0.02), "wo": _randn(g, (D, D), 0.02),
+                "w1": _randn(g, (2 * F, D), 0.02), "w2": _randn(g, (D, F), 0.02)}
+
+    if with_weights:
+        out["w_in"] = _randn(g, (D, 4 * C), 0.02)
+        out["w_out"] = _randn(g, (4 * C, D), 0.02)
+        out["mode_text"], out["mode_image"] = [], []
+        for _ in range(cfg.n_mode):
+            out["mode_text"].append(block_w())
+            out["mode_image"].append(block_w())
+        out["joint"] = [block_w() for _ in range(cfg.n_joint)]
+    out["mod_mode"] = _randn(g, (cfg.n_steps, cfg.n_mode, 2, 6, D), 0.1)
+    out["mod_joint"] = _randn(g, (cfg.n_steps, cfg.n_joint, 6, D), 0.1)
+    out["mod_final"] = _randn(g, (cfg.n_steps, 2, D), 0.1)
+    return out
