@@ -101,7 +101,7 @@ __device__ __forceinline__ void load_bf16x32(const uint16_t* src, float (&v)[32]
   if ((reinterpret_cast<uintptr_t>(src) & 31) == 0) {
 #pragma unroll
     for (int h = 0; h < 2; ++h)
-      asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      asm("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                    : "=r"(u[8 * h]), "=r"(u[8 * h + 1]), "=r"(u[8 * h + 2]), "=r"(u[8 * h + 3]), "=r"(u[8 * h + 4]),
                      "=r"(u[8 * h + 5]), "=r"(u[8 * h + 6]), "=r"(u[8 * h + 7])
                    : "l"(src + 16 * h));
@@ -204,10 +204,10 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
 #pragma unroll
           for (int g4 = 0; g4 < 4; ++g4) {
             float t[8];
-            asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=f"(t[0]), "=f"(t[1]), "=f"(t[2]), "=f"(t[3]), "=f"(t[4]), "=f"(t[5]), "=f"(t[6]),
-                           "=f"(t[7])
-                         : "l"(cs + (int64_t)g4 * p.M * 8));
+            // (not volatile: a read-only load the compiler may schedule early)
+            asm("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                : "=f"(t[0]), "=f"(t[1]), "=f"(t[2]), "=f"(t[3]), "=f"(t[4]), "=f"(t[5]), "=f"(t[6]), "=f"(t[7])
+                : "l"(cs + (int64_t)g4 * p.M * 8));
 #pragma unroll
             for (int u = 0; u < 4; ++u) {  // pair j0 + 4*g4 + u
               const int q = 4 * g4 + u;
