@@ -536,7 +536,8 @@ def run_dit(args):
              kl.rope_table(cfg.n_text, cfg.grid_h, cfg.grid_w, device=dev))
     ws = torch.empty(kl.dit_workspace_size(shape), dtype=torch.uint8, device=dev)
     w_abi = W.abi()
-    ts = [1.0 - i / cfg.n_steps for i in range(cfg.n_steps + 1)]
+    # flow-matching timesteps from 1 to 0, optionally time-shifted
+    ts = [args.shift * t / (1.0 + (args.shift - 1.0) * t) for t in (1.0 - i / cfg.n_steps for i in range(cfg.n_steps + 1))]
     mods = [(d["mod_mode"][i].contiguous(), d["mod_joint"][i].contiguous(), d["mod_final"][i].contiguous())
             for i in range(cfg.n_steps)]
     lat0 = d["latent"].contiguous()
@@ -570,7 +571,7 @@ def run_dit(args):
                                  "joint_blocks": cfg.n_joint, "tokens": cfg.n_text + cfg.grid_h * cfg.grid_w,
                                  "latent": [2 * cfg.grid_h, 2 * cfg.grid_w, cfg.channels],
                                  "block_calls_per_image": blocks_per_image,
-                                 "launch": "16 Euler steps captured in one CUDA graph"},
+                                 "launch": "16 Euler steps captured in one CUDA graph", "time_shift": args.shift},
                       "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin}), flush=True)
 
 
@@ -583,6 +584,7 @@ def main():
     ap.add_argument("--workload", default="t2i_1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dit", action="store_true", help="time the synthetic DiT loop instead (one JSON line)")
+    ap.add_argument("--shift", type=float, default=1.0, help="--dit: flow-matching time shift (1: linear)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

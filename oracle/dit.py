@@ -88,6 +88,15 @@ def dit_step(latent, text, weights, mods, shape, dt, attn="exact"):
     return euler(latent, v, dt, shape["grid_h"], shape["grid_w"], shape["channels"])
 
 
-def timesteps(n_steps):
-    """t_i = 1 - i/n, i = 0..n (linear, no shift)."""
-    return [1.0 - i / n_steps for i in range(n_steps + 1)]
+def timesteps(n_steps, shift=1.0):
+    """Flow-matching timesteps from t = 1 (noise) to t = 0: t_i = 1 - i/n,
+    mapped by the time shift s * t / (1 + (s - 1) * t) (s = 1: linear).  The
+    shift keeps the endpoints, is monotone and spends more steps at high
+    noise for s > 1 (the pages name a shift of 6.93 for the distilled
+    schedule: "black-forest-labs/flux-3-image-klein", Behavior and
+    constraints)."""
+    out = []
+    for i in range(n_steps + 1):
+        t = 1.0 - i / n_steps
+        out.append(shift * t / (1.0 + (shift - 1.0) * t))
+    return out

@@ -73,3 +73,17 @@ def test_velocity_is_finite_and_depends_on_the_text():
     u1 = dit.velocity(lat, text, w_nojoint, mods_nj, shape)
     u2 = dit.velocity(lat, text + 1.0, w_nojoint, mods_nj, shape)
     np.testing.assert_array_equal(u1, u2)
+
+
+def test_time_shift_keeps_endpoints_and_matches_its_closed_form():
+    lin = dit.timesteps(16)
+    sh = dit.timesteps(16, shift=6.93)
+    assert sh[0] == 1.0 and sh[-1] == 0.0
+    assert all(a > b for a, b in zip(sh, sh[1:]))  # strictly decreasing
+    # the shift maps t to s t / (1 + (s - 1) t): at t = 1/2 that is s / (s + 1)
+    assert abs(dit.timesteps(2, shift=6.93)[1] - 6.93 / 7.93) < 1e-15
+    # s = 1 is the linear schedule; s > 1 keeps every step at higher noise
+    assert dit.timesteps(16, shift=1.0) == lin
+    assert all(a >= b for a, b in zip(sh, lin))
+    # the Euler steps still integrate exactly from 1 to 0
+    assert abs(sum(b - a for a, b in zip(sh, sh[1:])) + 1.0) < 1e-15
