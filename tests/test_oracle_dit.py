@@ -4,6 +4,7 @@ exact special cases and the Euler closed form."""
 import numpy as np
 
 from oracle import dit
+from oracle.codecs import bf16_round
 from synth import DIT_CONFIGS, dit_inputs
 
 
@@ -87,3 +88,90 @@ def test_time_shift_keeps_endpoints_and_matches_its_closed_form():
     assert all(a >= b for a, b in zip(sh, lin))
     # the Euler steps still integrate exactly from 1 to 0
     assert abs(sum(b - a for a, b in zip(sh, sh[1:])) + 1.0) < 1e-15
+
+
+# ---------------------------------------------------------------- Cache-DiT
+
+
+def test_residual_diff_hand_values_and_special_cases():
+    # worked by hand: |1.5-1| + |-2+2| + |2-3| = 1.5 over |1| + |-2| + |3| = 6
+    assert dit.residual_diff([1.5, -2.0, 2.0], [1.0, -2.0, 3.0]) == 0.25
+    r_ref = np.array([[0.5, -1.0], [2.0, 0.0]])
+    assert dit.residual_diff(2 * r_ref, r_ref) == 1.0   # doubled residual: 100% change
+    assert dit.residual_diff(0 * r_ref, r_ref) == 1.0   # vanished residual
+    assert dit.residual_diff(r_ref, r_ref) == 0.0
+    assert dit.residual_diff(np.zeros(3), np.zeros(3)) == 0.0
+    assert dit.residual_diff(np.ones(3), np.zeros(3)) == float("inf")
+
+
+def _tiny_step_mods(step):
+    cfg = DIT_CONFIGS["dit_tiny"]
+    d = dit_inputs(cfg)
+    f = lambda t: t.float().numpy()
+    return {"mode": f(d["mod_mode"][step]), "joint": f(d["mod_joint"][step]), "final": f(d["mod_final"][step])}
+
+
+def test_cache_threshold_zero_reproduces_the_plain_steps():
+    cfg, lat, text, w, mods, shape = _tiny()
+    cache, plain = {}, lat.copy()
+    cached = lat.copy()
+    for step in range(cfg.n_steps):
+        m = _tiny_step_mods(step)
+        plain = dit.dit_step(plain, text, w, m, shape, -1 / 16)
+        cached = dit.dit_step(cached, text, w, m, shape, -1 / 16, cache=cache, threshold=0.0)
+        assert not cache["hit"]
+        np.testing.assert_array_equal(cached, plain)
+    assert cache["hits"] == 0
+
+
+def test_first_step_never_hits_and_a_repeated_input_reuses_exactly():
+    cfg, lat, text, w, mods, shape = _tiny()
+    cache = {}
+    v0 = dit.velocity_cached(lat, text, w, mods, shape, cache, threshold=float("inf"))
+    assert not cache["hit"] and cache["diff"] == float("inf")
+    np.testing.assert_array_equal(v0, dit.velocity(lat, text, w, mods, shape))
+    # the same input again: the probe residual is unchanged (diff 0), so the
+    # step skips the remaining blocks and bf16(F + (final - F)) = final exactly
+    v1 = dit.velocity_cached(lat, text, w, mods, shape, cache, threshold=1e-9)
+    assert cache["hit"] and cache["diff"] == 0.0 and cache["hits"] == 1
+    np.testing.assert_array_equal(v1, v0)
+
+
+def test_a_hit_keeps_the_reference_and_really_skips_the_rest():
+    cfg, lat, text, w, mods, shape = _tiny()
+    rng = np.random.default_rng(5)
+    lat_b = (lat + 0.05 * rng.standard_normal(lat.shape)).astype(np.float32)
+    lat_c = (lat + 0.10 * rng.standard_normal(lat.shape)).astype(np.float32)
+
+    def probe(x):
+        tok = dit._embed(x, text, w, shape)
+        f = dit._block(tok, 0, w, mods, shape, "exact")
+        return tok, f, f.astype(np.float64) - tok.astype(np.float64)
+
+    cache = {}
+    dit.velocity_cached(lat, text, w, mods, shape, cache, threshold=1e9)  # miss: reference A
+    _, _, r_a = probe(lat)
+    v_b = dit.velocity_cached(lat_b, text, w, mods, shape, cache, threshold=1e9)  # hit
+    assert cache["hit"]
+    tok_b, f_b, r_b = probe(lat_b)
+    assert cache["diff"] == dit.residual_diff(r_b, r_a) > 0
+    # the hit's velocity is the head on bf16(F_B + R_A), not the full stack's
+    full_b = dit.velocity(lat_b, text, w, mods, shape)
+    assert np.abs(v_b - full_b).max() > 0
+    _, f_a, _ = probe(lat)
+    final_a = f_a
+    for i in range(1, dit._n_blocks(w)):
+        final_a = dit._block(final_a, i, w, mods, shape, "exact")
+    r_rest_a = final_a.astype(np.float64) - f_a.astype(np.float64)
+    reuse = bf16_round(f_b.astype(np.float64) + r_rest_a)
+    np.testing.assert_array_equal(v_b, dit._head(reuse, w, mods, shape))
+    # step C is measured against A (the last full step), not against B
+    dit.velocity_cached(lat_c, text, w, mods, shape, cache, threshold=1e9)
+    _, _, r_c = probe(lat_c)
+    assert cache["diff"] == dit.residual_diff(r_c, r_a) != dit.residual_diff(r_c, r_b)
+    # a threshold below the change forces the full stack again, which then
+    # becomes the reference
+    v_c = dit.velocity_cached(lat_c, text, w, mods, shape, cache, threshold=0.0)
+    assert not cache["hit"]
+    np.testing.assert_array_equal(v_c, dit.velocity(lat_c, text, w, mods, shape))
+    np.testing.assert_array_equal(cache["r_ref"], r_c)
