@@ -542,10 +542,16 @@ def run_dit(args):
             for i in range(cfg.n_steps)]
     lat0 = d["latent"].contiguous()
     lat = lat0.clone()
+    # Cache-DiT: the skip of blocks 1.. is a conditional node in the graph
+    cache = kl.DitCache(shape, device=dev) if args.cache is not None else None
 
     def image():
         for i in range(cfg.n_steps):
-            kl.dit_step(shape, W, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i], workspace=ws, w_abi=w_abi)
+            if cache is None:
+                kl.dit_step(shape, W, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i], workspace=ws, w_abi=w_abi)
+            else:
+                kl.dit_step_cached(shape, W, cache, args.cache, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i],
+                                   workspace=ws, w_abi=w_abi)
 
     image()  # warm-up (eager)
     torch.cuda.synchronize()
@@ -555,6 +561,8 @@ def run_dit(args):
     times = []
     for _ in range(args.warmup + args.steps):
         lat.copy_(lat0)
+        if cache is not None:
+            cache.reset()  # a new generation
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         graph.replay()
@@ -565,6 +573,11 @@ def run_dit(args):
     st = kl.device_status()
     fin = bool(torch.isfinite(lat).all().item())
     blocks_per_image = cfg.n_steps * (2 * cfg.n_mode + cfg.n_joint)
+    extra = {}
+    if cache is not None:
+        h = cache.header()  # the last replay's generation
+        extra = {"cache_threshold": args.cache, "cached_steps_per_image": h["hits"], "steps_seen": h["steps"],
+                 "last_residual_diff": h["diff"]}
     print(json.dumps({"metric": "per-image DiT latency, synthetic 1024^2 T2I loop", "value": round(statistics.median(ms), 3),
                       "unit": "ms", "higher_is_better": False, "images": args.steps, "warmup": args.warmup,
                       "config": {"workload": cfg.name, "steps": cfg.n_steps, "per_mode_blocks": cfg.n_mode,
@@ -572,7 +585,7 @@ def run_dit(args):
                                  "latent": [2 * cfg.grid_h, 2 * cfg.grid_w, cfg.channels],
                                  "block_calls_per_image": blocks_per_image,
                                  "launch": "16 Euler steps captured in one CUDA graph", "time_shift": args.shift},
-                      "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin}), flush=True)
+                      "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin, **extra}), flush=True)
 
 
 def main():
@@ -585,6 +598,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dit", action="store_true", help="time the synthetic DiT loop instead (one JSON line)")
     ap.add_argument("--shift", type=float, default=1.0, help="--dit: flow-matching time shift (1: linear)")
+    ap.add_argument("--cache", type=float, default=None,
+                    help="--dit: Cache-DiT residual-difference threshold (e.g. 0.24); default off")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

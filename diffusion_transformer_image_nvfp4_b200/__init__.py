@@ -86,6 +86,11 @@ class _DitStepIO(ctypes.Structure):
                 ("rope_image", ctypes.c_void_p), ("rope_joint", ctypes.c_void_p), ("dt", ctypes.c_float)]
 
 
+class _DitCacheHeader(ctypes.Structure):
+    _fields_ = [("num", ctypes.c_double), ("den", ctypes.c_double), ("diff", ctypes.c_float), ("hit", ctypes.c_int),
+                ("has_ref", ctypes.c_int), ("hits", ctypes.c_int), ("steps", ctypes.c_int)]
+
+
 _LIB = None
 _VP, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 _SIGS = {
@@ -110,6 +115,10 @@ _SIGS = {
     "kl_dit_workspace_size": ([ctypes.POINTER(_DitShape)], _SZ),
     "kl_dit_step": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitWeights), ctypes.POINTER(_DitStepIO), _VP, _SZ,
                      _VP], _I),
+    "kl_dit_cache_size": ([ctypes.POINTER(_DitShape)], _SZ),
+    "kl_dit_cache_reset": ([_VP, _VP], _I),
+    "kl_dit_step_cached": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitWeights), ctypes.POINTER(_DitStepIO),
+                            ctypes.c_float, _VP, _SZ, _VP, _SZ, _VP], _I),
 }
 
 
@@ -406,6 +415,64 @@ def dit_step(shape, weights, latent, text, mod_mode, mod_joint, mod_final, rope_
                     rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt))
     _check(lib().kl_dit_step(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
                              workspace.numel(), _stream()), "kl_dit_step")
+    return latent
+
+
+class DitCache:
+    """Device state of kl_dit_step_cached (Cache-DiT) for one generation:
+    a kl_dit_cache_header followed by F bf16 [T, D], r_cur, r_ref and R fp32
+    [T, D], each at a 256-byte boundary.  reset() before every generation."""
+
+    def __init__(self, shape, device=None):
+        sh = shape.abi()
+        n = lib().kl_dit_cache_size(ctypes.byref(sh))
+        if n == 0:
+            raise KLError(2, "kl_dit_cache_size")
+        self.shape = shape
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+        self.reset()
+
+    def reset(self):
+        _check(lib().kl_dit_cache_reset(self.buf.data_ptr(), _stream()), "kl_dit_cache_reset")
+
+    def header(self):
+        """The header as a dict (copies it to the host: synchronising)."""
+        raw = bytes(self.buf[:ctypes.sizeof(_DitCacheHeader)].cpu().numpy().tobytes())
+        h = _DitCacheHeader.from_buffer_copy(raw)
+        return {f: getattr(h, f) for f, _ in _DitCacheHeader._fields_}
+
+    def arrays(self):
+        """Views F (bf16), r_cur, r_ref, R (fp32), each [T, D]."""
+        s = self.shape
+        n = (s.n_text + s.grid_h * s.grid_w) * s.D
+        up = lambda b: (b + 255) // 256 * 256
+        off = up(ctypes.sizeof(_DitCacheHeader))
+        out = {}
+        for name, dt, es in (("F", torch.bfloat16, 2), ("r_cur", torch.float32, 4), ("r_ref", torch.float32, 4),
+                             ("R", torch.float32, 4)):
+            out[name] = self.buf[off:off + n * es].view(dt).view(-1, s.D)
+            off += up(n * es)
+        return out
+
+
+def dit_step_cached(shape, weights, cache, threshold, latent, text, mod_mode, mod_joint, mod_final, rope_text,
+                    rope_image, rope_joint, dt, workspace=None, w_abi=None):
+    """kl_dit_step_cached: dit_step with Cache-DiT step caching at
+    ``threshold`` (the residual-difference threshold; 0 never reuses), state
+    in ``cache`` (a DitCache).  Eager calls synchronise the stream once to read
+    the decision; under CUDA graph capture the decision stays on the device."""
+    _need(latent, torch.float32, "latent")
+    _need(text, torch.bfloat16, "text")
+    sh = shape.abi()
+    need = lib().kl_dit_workspace_size(ctypes.byref(sh))
+    if workspace is None:
+        workspace = _workspace(need, latent.device, "dit")
+    w = weights.abi() if w_abi is None else w_abi
+    io = _DitStepIO(latent.data_ptr(), text.data_ptr(), _ptr(mod_mode), _ptr(mod_joint), mod_final.data_ptr(),
+                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt))
+    _check(lib().kl_dit_step_cached(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), float(threshold),
+                                    cache.buf.data_ptr(), cache.buf.numel(), workspace.data_ptr(), workspace.numel(),
+                                    _stream()), "kl_dit_step_cached")
     return latent
 
 

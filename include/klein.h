@@ -390,6 +390,56 @@ size_t kl_dit_workspace_size(const kl_dit_shape* shape);
 kl_status kl_dit_step(const kl_dit_shape* shape, const kl_dit_weights* w, const kl_dit_step_io* io,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * kl_dit_step_cached -- kl_dit_step with Cache-DiT step caching ([P1]
+ * "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs", How it
+ * works: a residual difference between denoising steps is watched and, under
+ * a threshold, cached transformer outputs are reused; What you can do:
+ * residual_diff_threshold 0.24).  Readings (the pages give no more):
+ *   block 0 of the stack (the first per-mode pair, else the first joint
+ *     block) is the probe and runs every step: F = its output, r = F - its
+ *     input (fp32 of the bf16 tokens, all T = n_text + grid_h*grid_w rows);
+ *   diff = sum|r - r_ref| / sum|r_ref| (0/0 -> 0, x/0 -> +inf), r_ref being
+ *     the probe residual of the last step that ran every block; no
+ *     reference yet (first step after kl_dit_cache_reset) -> diff = +inf;
+ *   hit = diff < threshold: blocks 1.. are skipped and the final tokens are
+ *     bf16(F + R); miss: blocks 1.. run, R = final - F (fp32) and r_ref = r;
+ *   the head (final LN, adaLN, w_out, Euler update) runs either way.
+ * The sums are fp32 per thread and fp64 across thread blocks (their order is
+ * not fixed, so diff may vary in its last bits between runs); the decision
+ * compares diff in fp64.
+ *
+ * cache: a caller-owned device buffer of kl_dit_cache_size(shape) bytes,
+ * 256-byte aligned, holding a kl_dit_cache_header at offset 0 followed by
+ * F bf16 [T, D], r_cur fp32 [T, D], r_ref fp32 [T, D], R fp32 [T, D], each at
+ * the next 256-byte boundary.  Call kl_dit_cache_reset(cache, stream) before
+ * the first step of every generation (it also creates, outside any graph
+ * capture, the side stream used below).  The header can be read back (e.g.
+ * with cudaMemcpy) after a step: diff, hit, and hits / steps since the reset.
+ *
+ * Outside stream capture the call synchronises the stream once, to read the
+ * decision on the host.  Under capture (a CUDA graph) it does not: a one-
+ * thread kernel takes the decision on the device and sets the condition of a
+ * conditional (IF) graph node whose body, captured on a side stream, holds
+ * blocks 1..; a skipped step then costs the probe block, the head and three
+ * small kernels.  Errors: as kl_dit_step; KL_ERR_UNSUPPORTED_SHAPE without any
+ * block; KL_ERR_WORKSPACE if cache_bytes is too small.
+ */
+typedef struct kl_dit_cache_header {
+  double num, den; /* sums of the step in flight (zero between steps) */
+  float diff;      /* residual difference of the last step (+inf: no reference) */
+  int hit;         /* 1: the last step reused the cache */
+  int has_ref;     /* 1: a reference step exists */
+  int hits;        /* hits since the last reset */
+  int steps;       /* steps since the last reset */
+} kl_dit_cache_header;
+
+size_t kl_dit_cache_size(const kl_dit_shape* shape); /* 0: bad shape or no block */
+kl_status kl_dit_cache_reset(void* cache, void* stream);
+kl_status kl_dit_step_cached(const kl_dit_shape* shape, const kl_dit_weights* w, const kl_dit_step_io* io,
+                             float threshold, void* cache, size_t cache_bytes, void* workspace, size_t ws_bytes,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

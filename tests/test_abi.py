@@ -107,3 +107,30 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kl, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         kl.lib()
+
+
+def test_dit_cache_size_and_cached_step_validation(L):
+    up = lambda b: (b + 255) // 256 * 256
+    assert ctypes.sizeof(kl._DitCacheHeader) == 40
+    sh = kl._DitShape(16, 4, 4, 32, 128, 1, 384, 1, 2, 1)
+    T, D = 16 + 4 * 4, 128
+    # header, then F bf16 and r_cur, r_ref, R fp32, each [T, D] at 256-byte boundaries
+    assert L.kl_dit_cache_size(ctypes.byref(sh)) == 256 + up(T * D * 2) + 3 * up(T * D * 4)
+    none = kl._DitShape(16, 4, 4, 32, 128, 1, 384, 0, 0, 1)
+    assert L.kl_dit_cache_size(ctypes.byref(none)) == 0
+    fake = 1 << 20   # never dereferenced: every call below fails validation first
+    t = kl._NVFP4Tensor(fake, fake, fake)
+    blocks = (kl._BlockWeights * 2)(kl._BlockWeights(t, t, t, t), kl._BlockWeights(t, t, t, t))
+    bp = ctypes.cast(blocks, ctypes.POINTER(kl._BlockWeights))
+    w = kl._DitWeights(t, bp, bp, bp, t)
+    io = kl._DitStepIO(fake, fake, fake, fake, fake, fake, fake, fake, -0.0625)
+    ws = L.kl_dit_workspace_size(ctypes.byref(sh))
+    need = L.kl_dit_cache_size(ctypes.byref(sh))
+    step = lambda shape, cache, nbytes: L.kl_dit_step_cached(ctypes.byref(shape), ctypes.byref(w), ctypes.byref(io),
+                                                             0.24, cache, nbytes, fake, ws, None)
+    assert step(sh, None, need) == 1           # no cache
+    assert step(sh, fake, need - 1) == 4       # cache too small
+    assert step(sh, fake + 16, need) == 3      # cache not 256-byte aligned
+    assert step(none, fake, need) == 2         # no block to probe
+    assert L.kl_dit_cache_reset(None, None) == 1
+    assert L.kl_dit_cache_reset(fake + 8, None) == 3
