@@ -523,7 +523,7 @@ def run_dit(args):
     cfg = DIT_CONFIGS["dit_t2i_1024"]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    d = dit_inputs(cfg, device=dev)
+    d = dit_inputs(cfg, device=dev, mods=args.mods)
     blocks = lambda bl: [kl.prepare_block_weights(b["wqkv"], b["wo"], b["w1"], b["w2"]) for b in bl]
     W = kl.DitWeights(kl.quantize_nvfp4(d["w_in"]), blocks(d["mode_text"]), blocks(d["mode_image"]),
                       blocks(d["joint"]), kl.quantize_nvfp4(d["w_out"]))
@@ -584,7 +584,8 @@ def run_dit(args):
                                  "joint_blocks": cfg.n_joint, "tokens": cfg.n_text + cfg.grid_h * cfg.grid_w,
                                  "latent": [2 * cfg.grid_h, 2 * cfg.grid_w, cfg.channels],
                                  "block_calls_per_image": blocks_per_image,
-                                 "launch": "16 Euler steps captured in one CUDA graph", "time_shift": args.shift},
+                                 "launch": "16 Euler steps captured in one CUDA graph", "time_shift": args.shift,
+                                 "modulations": args.mods},
                       "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin, **extra}), flush=True)
 
 
@@ -600,6 +601,8 @@ def main():
     ap.add_argument("--shift", type=float, default=1.0, help="--dit: flow-matching time shift (1: linear)")
     ap.add_argument("--cache", type=float, default=None,
                     help="--dit: Cache-DiT residual-difference threshold (e.g. 0.24); default off")
+    ap.add_argument("--mods", choices=("independent", "smooth"), default="independent",
+                    help="--dit: modulations drawn per step, or smooth in t (m0 + t m1)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -133,15 +133,18 @@ DIT_CONFIGS = {
 }
 
 
-def dit_inputs(cfg, with_weights=True, device="cpu"):
+def dit_inputs(cfg, with_weights=True, device="cpu", mods="independent"):
     """Seeded inputs of a DiT run as CPU tensors.  Draw order: latent (fp32
     N(0,1)); text (bf16 N(0,1)); w_in [D, 4C], w_out [4C, D] (N(0,0.02));
     per-mode blocks i = 0..n_mode-1: text weights then image weights (each
     Wqkv, Wo, W1, W2 as in block_inputs); joint blocks; modulation vectors
-    (N(0,0.1)): mode [n_mode, 2, 6, D], joint [n_joint, 6, D], final [2, D]
-    for each of the n_steps steps ([n_steps, ...]).  ``device``: where the
-    generator and tensors live (a CUDA generator draws different numbers than
-    the CPU one; the parity tests use the CPU draws)."""
+    (N(0,0.1)): mode [n_mode, 2, 6, D], joint [n_joint, 6, D], final [2, D].
+    ``mods="independent"``: drawn afresh for each of the n_steps steps
+    ([n_steps, ...]); ``mods="smooth"``: two such sets m0 then m1 are drawn and
+    step i takes bf16(m0 + t_i m1) with t_i = 1 - i / n_steps, a stand-in for
+    modulations that a timestep embedding makes a smooth function of t.
+    ``device``: where the generator and tensors live (a CUDA generator draws
+    different numbers than the CPU one; the parity tests use the CPU draws)."""
     if isinstance(cfg, str):
         cfg = DIT_CONFIGS[cfg]
     g = torch.Generator(device=device).manual_seed(cfg.seed)
@@ -166,7 +169,16 @@ def dit_inputs(cfg, with_weights=True, device="cpu"):
             out["mode_text"].append(block_w())
             out["mode_image"].append(block_w())
         out["joint"] = [block_w() for _ in range(cfg.n_joint)]
-    out["mod_mode"] = _randn(g, (cfg.n_steps, cfg.n_mode, 2, 6, D), 0.1)
-    out["mod_joint"] = _randn(g, (cfg.n_steps, cfg.n_joint, 6, D), 0.1)
-    out["mod_final"] = _randn(g, (cfg.n_steps, 2, D), 0.1)
+    shapes = {"mod_mode": (cfg.n_mode, 2, 6, D), "mod_joint": (cfg.n_joint, 6, D), "mod_final": (2, D)}
+    if mods == "independent":
+        for k, sh in shapes.items():
+            out[k] = _randn(g, (cfg.n_steps,) + sh, 0.1)
+    elif mods == "smooth":
+        m0 = {k: _randn(g, sh, 0.1).float() for k, sh in shapes.items()}
+        m1 = {k: _randn(g, sh, 0.1).float() for k, sh in shapes.items()}
+        t = [1.0 - i / cfg.n_steps for i in range(cfg.n_steps)]
+        for k in shapes:
+            out[k] = torch.stack([m0[k] + ti * m1[k] for ti in t]).to(torch.bfloat16)
+    else:
+        raise ValueError("mods must be 'independent' or 'smooth'")
     return out

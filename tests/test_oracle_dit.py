@@ -175,3 +175,23 @@ def test_a_hit_keeps_the_reference_and_really_skips_the_rest():
     assert not cache["hit"]
     np.testing.assert_array_equal(v_c, dit.velocity(lat_c, text, w, mods, shape))
     np.testing.assert_array_equal(cache["r_ref"], r_c)
+
+
+def test_smooth_modulations_are_linear_in_t_and_keep_the_other_draws():
+    from synth import DitConfig
+    cfg = DitConfig("smooth_probe", 16, 4, 4, 32, 128, 1, 384, 1, 2, 8, "bf16", 7)
+    ind = dit_inputs(cfg, with_weights=False)
+    smo = dit_inputs(cfg, with_weights=False, mods="smooth")
+    np.testing.assert_array_equal(ind["latent"].numpy(), smo["latent"].numpy())
+    np.testing.assert_array_equal(ind["text"].float().numpy(), smo["text"].float().numpy())
+    for k in ("mod_mode", "mod_joint", "mod_final"):
+        m = smo[k].double().numpy()
+        assert m.shape == ind[k].shape
+        # equal t steps: second differences vanish up to the three bf16
+        # roundings in them (8 significant bits: each within 2^-8 of its value)
+        second = m[2:] - 2 * m[1:-1] + m[:-2]
+        assert np.abs(second).max() <= 4 * 2.0 ** -8 * np.abs(m).max()
+        # consecutive steps move by |m1| / n_steps, far less than fresh draws
+        step = np.abs(np.diff(m, axis=0)).mean()
+        fresh = np.abs(np.diff(ind[k].double().numpy(), axis=0)).mean()
+        assert step < 0.2 * fresh
