@@ -547,11 +547,13 @@ def run_dit(args):
 
     def image():
         for i in range(cfg.n_steps):
+            tau = args.sol_tau if i >= args.sol_dense_steps else 0.0  # Sol-Attention after the dense steps
             if cache is None:
-                kl.dit_step(shape, W, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i], workspace=ws, w_abi=w_abi)
+                kl.dit_step(shape, W, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i], workspace=ws, w_abi=w_abi,
+                            sol_tau=tau)
             else:
                 kl.dit_step_cached(shape, W, cache, args.cache, lat, d["text"], *mods[i], *ropes, ts[i + 1] - ts[i],
-                                   workspace=ws, w_abi=w_abi)
+                                   workspace=ws, w_abi=w_abi, sol_tau=tau)
 
     image()  # warm-up (eager)
     torch.cuda.synchronize()
@@ -585,8 +587,68 @@ def run_dit(args):
                                  "latent": [2 * cfg.grid_h, 2 * cfg.grid_w, cfg.channels],
                                  "block_calls_per_image": blocks_per_image,
                                  "launch": "16 Euler steps captured in one CUDA graph", "time_shift": args.shift,
-                                 "modulations": args.mods},
+                                 "modulations": args.mods, "sol_tau": args.sol_tau,
+                                 "sol_dense_steps": args.sol_dense_steps},
                       "min_ms": round(min(ms), 3), "device_status": st, "latent_finite": fin, **extra}), flush=True)
+
+
+def run_sol(args):
+    """Sol-Attention at the 1024^2 T2I attention shape (4,608 tokens, 24
+    heads, FP8): device time of key-tile selection + sparse attention against
+    dense attention, on seeded inputs with tile structure (synth
+    sparse_attention_qkv), inputs resident, L2 flushed between steps."""
+    import diffusion_transformer_image_nvfp4_b200 as kl
+    from synth import sparse_attention_qkv
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, H = 4608, 24
+    D = H * 128
+    qkv = sparse_attention_qkv(T, H, seed=5).to(dev)
+    amax = qkv.float().abs().view(T, 3, H, 128).amax(dim=(0, 3)).reshape(-1).contiguous()
+    x8, sc = kl.cast_fp8_per_head(qkv, amax)
+    q, k, v = x8, x8[:, D:], x8[:, 2 * D:]
+    scales = dict(sq=sc[:H], sk=sc[H:2 * H], sv=sc[2 * H:])
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def sparse_step():
+        lst = kl.sol_select(q, k, T, H, 3 * D, args.sol, "fp8", sq=scales["sq"], sk=scales["sk"])
+        kl.joint_attention_sparse(q, k, v, T, H, 3 * D, lst, "fp8", out=out, **scales)
+        return lst
+
+    def dense_step():
+        kl.joint_attention(q, k, v, T, H, 3 * D, "fp8", out=out, **scales)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ms.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in ms])
+
+    lst = sparse_step()
+    torch.cuda.synchronize()
+    nkt = -(-T // 128)
+    kept = float(lst[:, :, 0].float().mean().item()) / nkt
+    t_sparse, t_dense = timed(sparse_step), timed(dense_step)
+    flops_dense = 4.0 * T * T * H * 128
+    print(json.dumps({"metric": "Sol-Attention device time (selection + sparse FP8 attention), 1024^2 T2I shape",
+                      "value": round(t_sparse * 1000, 1), "unit": "us", "higher_is_better": False,
+                      "dense_us": round(t_dense * 1000, 1), "speedup": round(t_dense / t_sparse, 3),
+                      "kept_tile_fraction": round(kept, 4), "tau": args.sol,
+                      "kept_work_tflops": round(flops_dense * kept / (t_sparse * 1e-3) / 1e12, 1),
+                      "config": {"workload": "sol_attention_t2i_1024", "tokens": T, "heads": H, "query_block": 256,
+                                 "key_tile": 128, "inputs": "synth.sparse_attention_qkv(seed 5)",
+                                 "l2": "flushed between timed steps (256 MiB write, outside the timed events)"},
+                      "steps": args.steps, "warmup": args.warmup, "device_status": kl.device_status()}), flush=True)
 
 
 def main():
@@ -601,6 +663,10 @@ def main():
     ap.add_argument("--shift", type=float, default=1.0, help="--dit: flow-matching time shift (1: linear)")
     ap.add_argument("--cache", type=float, default=None,
                     help="--dit: Cache-DiT residual-difference threshold (e.g. 0.24); default off")
+    ap.add_argument("--sol", type=float, default=None,
+                    help="time Sol-Attention (selection + sparse attention) at this tau against dense attention")
+    ap.add_argument("--sol-tau", type=float, default=0.0, help="--dit: Sol-Attention tau for every block (0: dense)")
+    ap.add_argument("--sol-dense-steps", type=int, default=0, help="--dit: the first N steps stay dense")
     ap.add_argument("--mods", choices=("independent", "smooth"), default="independent",
                     help="--dit: modulations drawn per step, or smooth in t (m0 + t m1)")
     args = ap.parse_args()
@@ -609,6 +675,9 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.dit:
         run_dit(args)
+        return
+    if args.sol is not None:
+        run_sol(args)
         return
     if args.impl == "reference":
         run_reference(args, wl)

@@ -65,7 +65,7 @@ class _BlockIO(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("mod", ctypes.c_void_p * 6), ("rope_cs", ctypes.c_void_p),
                 ("T", ctypes.c_int64), ("D", ctypes.c_int64), ("H", ctypes.c_int64), ("F", ctypes.c_int64),
                 ("attn_precision", ctypes.c_int), ("out", ctypes.c_void_p),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("sol_tau", ctypes.c_float)]
 
 
 class _DitShape(ctypes.Structure):
@@ -83,7 +83,8 @@ class _DitWeights(ctypes.Structure):
 class _DitStepIO(ctypes.Structure):
     _fields_ = [("latent", ctypes.c_void_p), ("text", ctypes.c_void_p), ("mod_mode", ctypes.c_void_p),
                 ("mod_joint", ctypes.c_void_p), ("mod_final", ctypes.c_void_p), ("rope_text", ctypes.c_void_p),
-                ("rope_image", ctypes.c_void_p), ("rope_joint", ctypes.c_void_p), ("dt", ctypes.c_float)]
+                ("rope_image", ctypes.c_void_p), ("rope_joint", ctypes.c_void_p), ("dt", ctypes.c_float),
+                ("sol_tau", ctypes.c_float)]
 
 
 class _DitCacheHeader(ctypes.Structure):
@@ -110,6 +111,11 @@ _SIGS = {
     "kl_rope_table": ([ctypes.POINTER(_TokenLayout), ctypes.c_float, _VP, _VP], _I),
     "kl_cast_fp8_per_head": ([_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP], _I),
     "kl_joint_attention_fp8": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _I64, _I64, _I64, _I, _VP, _VP, _VP], _I),
+    "kl_sol_list_ints": ([_I64, _I64, _I], _SZ),
+    "kl_sol_workspace_size": ([_I64, _I64, _I], _SZ),
+    "kl_sol_select": ([_VP, _VP, _I64, _VP, _VP, _I64, _I64, _I, ctypes.c_float, _VP, _VP, _SZ, _VP], _I),
+    "kl_joint_attention_sparse": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _I64, _I64, _I64, _I, _VP, _VP, _VP, _VP],
+                                  _I),
     "kl_block_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
     "kl_joint_block_forward": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
     "kl_dit_workspace_size": ([ctypes.POINTER(_DitShape)], _SZ),
@@ -299,6 +305,37 @@ def joint_attention(q, k, v, T, H, ld, precision="fp8", sq=None, sk=None, sv=Non
     return out
 
 
+SOL_QUERY_ROWS = {"fp8": 256, "bf16": 128}
+
+
+def sol_select(q, k, T, H, ld, tau, precision="fp8", sq=None, sk=None):
+    """kl_sol_select: Sol-Attention key-tile lists (int32 [H, n_qb, n_kt + 1]:
+    count, then the kept tile indices in ascending order)."""
+    n = lib().kl_sol_list_ints(T, H, ATTN[precision])
+    nqb = -(-T // SOL_QUERY_ROWS[precision])
+    nkt = -(-T // 128)
+    assert n == H * nqb * (nkt + 1)
+    lst = torch.zeros(n, dtype=torch.int32, device=q.device)
+    need = lib().kl_sol_workspace_size(T, H, ATTN[precision])
+    ws = _workspace(need, q.device, "sol")
+    _check(lib().kl_sol_select(q.data_ptr(), k.data_ptr(), ld, _ptr(sq), _ptr(sk), T, H, ATTN[precision], float(tau),
+                               lst.data_ptr(), ws.data_ptr(), ws.numel(), _stream()), "kl_sol_select")
+    return lst.view(H, nqb, nkt + 1)
+
+
+def joint_attention_sparse(q, k, v, T, H, ld, kv_list, precision="fp8", sq=None, sk=None, sv=None, amax=None,
+                           out=None):
+    """kl_joint_attention_sparse: joint_attention over the key tiles of
+    ``kv_list`` (the layout sol_select returns)."""
+    if out is None:
+        out = torch.empty((T, H * 128), dtype=torch.bfloat16, device=q.device)
+    _need(kv_list, torch.int32, "kv_list")
+    _check(lib().kl_joint_attention_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), ld, _ptr(sq), _ptr(sk),
+                                           _ptr(sv), T, H, 128, ATTN[precision], kv_list.data_ptr(), out.data_ptr(),
+                                           _ptr(amax), _stream()), "kl_joint_attention_sparse")
+    return out
+
+
 # ---------------------------------------------------------------- block
 @dataclass
 class BlockWeights:
@@ -325,11 +362,13 @@ BLOCK_STAGES = ("ln1", "qkv_gemm", "fp8_cast", "attention", "quant_o", "out_gemm
                 "quant_h", "mlp_down_gemm")
 
 
-def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, workspace=None, stage_events=None):
+def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, workspace=None, stage_events=None,
+                        sol_tau=0.0):
     """kl_joint_block_forward.  ``mod`` maps shift1, scale1, gate1, shift2,
     scale2, gate2 to bf16 [D] CUDA tensors.  ``stage_events`` (optional): a list
     of len(BLOCK_STAGES)+1 recorded torch.cuda.Event(enable_timing=True); the
-    library re-records them around each stage on the current stream."""
+    library re-records them around each stage on the current stream.
+    ``sol_tau`` > 0: Sol-Attention tile skipping at that threshold."""
     _need(x, torch.bfloat16, "x")
     T, D = x.shape
     names = ("shift1", "scale1", "gate1", "shift2", "scale2", "gate2")
@@ -346,7 +385,8 @@ def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, wo
             raise ValueError("stage_events: need one event per stage plus one")
         ev = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
     io = _BlockIO(x.data_ptr(), (ctypes.c_void_p * 6)(*[mod[n].data_ptr() for n in names]), rope_cs.data_ptr(),
-                  T, D, H, F, ATTN[attn], out.data_ptr(), ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)))
+                  T, D, H, F, ATTN[attn], out.data_ptr(), ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)),
+                  float(sol_tau))
     w = weights.abi()
     _check(lib().kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(), workspace.numel(),
                                         _stream()), "kl_joint_block_forward")
@@ -398,7 +438,7 @@ def dit_workspace_size(shape):
 
 
 def dit_step(shape, weights, latent, text, mod_mode, mod_joint, mod_final, rope_text, rope_image, rope_joint, dt,
-             workspace=None, w_abi=None):
+             workspace=None, w_abi=None, sol_tau=0.0):
     """kl_dit_step: one Euler step, latent (fp32 [2gh, 2gw, C], CUDA) updated in
     place.  mod_mode bf16 [n_mode, 2, 6, D]; mod_joint bf16 [n_joint, 6, D];
     mod_final bf16 [2, D]; rope tables from rope_table for the text-only,
@@ -412,7 +452,7 @@ def dit_step(shape, weights, latent, text, mod_mode, mod_joint, mod_final, rope_
         workspace = _workspace(need, latent.device, "dit")
     w = weights.abi() if w_abi is None else w_abi
     io = _DitStepIO(latent.data_ptr(), text.data_ptr(), _ptr(mod_mode), _ptr(mod_joint), mod_final.data_ptr(),
-                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt))
+                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt), float(sol_tau))
     _check(lib().kl_dit_step(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
                              workspace.numel(), _stream()), "kl_dit_step")
     return latent
@@ -456,7 +496,7 @@ class DitCache:
 
 
 def dit_step_cached(shape, weights, cache, threshold, latent, text, mod_mode, mod_joint, mod_final, rope_text,
-                    rope_image, rope_joint, dt, workspace=None, w_abi=None):
+                    rope_image, rope_joint, dt, workspace=None, w_abi=None, sol_tau=0.0):
     """kl_dit_step_cached: dit_step with Cache-DiT step caching at
     ``threshold`` (the residual-difference threshold; 0 never reuses), state
     in ``cache`` (a DitCache).  Eager calls synchronise the stream once to read
@@ -469,7 +509,7 @@ def dit_step_cached(shape, weights, cache, threshold, latent, text, mod_mode, mo
         workspace = _workspace(need, latent.device, "dit")
     w = weights.abi() if w_abi is None else w_abi
     io = _DitStepIO(latent.data_ptr(), text.data_ptr(), _ptr(mod_mode), _ptr(mod_joint), mod_final.data_ptr(),
-                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt))
+                    rope_text.data_ptr(), rope_image.data_ptr(), rope_joint.data_ptr(), float(dt), float(sol_tau))
     _check(lib().kl_dit_step_cached(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), float(threshold),
                                     cache.buf.data_ptr(), cache.buf.numel(), workspace.data_ptr(), workspace.numel(),
                                     _stream()), "kl_dit_step_cached")

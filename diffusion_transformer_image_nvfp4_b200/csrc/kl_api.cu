@@ -318,6 +318,64 @@ kl_status kl_joint_attention_fp8(const void* q, const void* k, const void* v, in
   return e == cudaSuccess ? KL_OK : cuda_fail(e);
 }
 
+size_t kl_sol_list_ints(int64_t T, int64_t H, int precision) {
+  if (T < 1 || H < 1 || (precision != KL_ATTN_FP8 && precision != KL_ATTN_BF16)) return 0;
+  return sol_list_ints(T, H, precision == KL_ATTN_FP8);
+}
+
+size_t kl_sol_workspace_size(int64_t T, int64_t H, int precision) {
+  if (T < 1 || H < 1 || (precision != KL_ATTN_FP8 && precision != KL_ATTN_BF16)) return 0;
+  return sol_workspace_bytes(T, H, precision == KL_ATTN_FP8);
+}
+
+kl_status kl_sol_select(const void* q, const void* k, int64_t ld, const float* sq, const float* sk, int64_t T,
+                        int64_t H, int precision, float tau, int* kv_list, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  if (!q || !k || !kv_list) return KL_ERR_INVALID_ARG;
+  if (precision != KL_ATTN_FP8 && precision != KL_ATTN_BF16) return KL_ERR_INVALID_ARG;
+  if (precision == KL_ATTN_FP8 && (!sq || !sk)) return KL_ERR_INVALID_ARG;
+  if (!(tau >= 0.f)) return KL_ERR_INVALID_ARG;  // also rejects NaN
+  if (T < 1 || H < 1 || H > 65535 || ld < H * 128 || (T + 127) / 128 > 48 * 1024) return KL_ERR_UNSUPPORTED_SHAPE;
+  const bool fp8 = precision == KL_ATTN_FP8;
+  if (!workspace || ws_bytes < sol_workspace_bytes(T, H, fp8)) return KL_ERR_WORKSPACE;
+  if (!aligned(kv_list, 4) || !aligned(workspace, 16)) return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  cudaError_t e = launch_sol_select(q, k, ld, sq, sk, T, H, fp8, tau, kv_list, workspace,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
+kl_status kl_joint_attention_sparse(const void* q, const void* k, const void* v, int64_t ld, const float* sq,
+                                    const float* sk, const float* sv, int64_t T, int64_t H, int64_t head_dim,
+                                    int precision, const int* kv_list, void* out, float* amax_out, void* stream) {
+  if (!q || !k || !v || !out || !kv_list) return KL_ERR_INVALID_ARG;
+  if (precision != KL_ATTN_FP8 && precision != KL_ATTN_BF16) return KL_ERR_INVALID_ARG;
+  if (precision == KL_ATTN_FP8 && (!sq || !sk || !sv)) return KL_ERR_INVALID_ARG;
+  if (head_dim != 128 || T < 1 || H < 1 || H > 65535 || T > (int64_t)1 << 31 || ld < H * 128 || ld % 64)
+    return KL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(kv_list, 4))
+    return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  AttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.ld = ld;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.T = T;
+  a.H = H;
+  a.fp8 = precision == KL_ATTN_FP8;
+  a.out = out;
+  a.amax = amax_out;
+  a.kv_list = kv_list;
+  cudaError_t e = launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------ block driver
 // Workspace layout (each piece 256-byte aligned):
 //   words  : amax[0..3] (O at 1, h at 3), gs[4..7], qkv amax [3H], fp8 scales [3H],
@@ -335,6 +393,8 @@ struct BlockWs {
   float2* stats;
   uint8_t *acodes, *ascales, *qkv8, *hcodes, *hscales;
   uint16_t *qkv, *o, *x1, *h;
+  void* sol_ws;   // Sol-Attention block means
+  int* sol_list;  // Sol-Attention key-tile lists
   size_t total;
 };
 static BlockWs block_ws_layout(uint8_t* base, int64_t T, int64_t D, int64_t H, int64_t F, int prec) {
@@ -357,6 +417,8 @@ static BlockWs block_ws_layout(uint8_t* base, int64_t T, int64_t D, int64_t H, i
   w.h = reinterpret_cast<uint16_t*>(take((size_t)T * F * 2));
   w.hcodes = take((size_t)T * F / 2);
   w.hscales = take((size_t)Tp * F / 16);
+  w.sol_ws = take(sol_workspace_bytes(T, H, prec == KL_ATTN_FP8));
+  w.sol_list = reinterpret_cast<int*>(take(sol_list_ints(T, H, prec == KL_ATTN_FP8) * sizeof(int)));
   w.total = off;
   return w;
 }
@@ -452,6 +514,10 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
     a.v = ws.qkv + 2 * D;
   }
   mark(3);
+  if (io->sol_tau > 0.f) {  // Sol-Attention: the key tiles each query block visits
+    KL_TRY(launch_sol_select(a.q, a.k, a.ld, a.sq, a.sk, T, H, a.fp8 != 0, io->sol_tau, ws.sol_list, ws.sol_ws, s));
+    a.kv_list = ws.sol_list;
+  }
   KL_TRY(launch_attention(a, s));
   mark(4);
   // 5. O -> NVFP4 (gs from the attention amax)

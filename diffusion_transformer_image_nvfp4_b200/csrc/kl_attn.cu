@@ -29,6 +29,12 @@
 //    p * P_SCALE, and the halves' sums are added once at the end.
 //    Finally O = O_tmem / l (FP8: times s_v), bf16, and a tensor amax.
 // TMEM per query tile: S [128 cols] + O [128 cols].
+//
+// Sol-Attention ([P1] How it works: less important token pairs are skipped
+// by a sparsity threshold): with a key-tile list (kl_sol_select) each CTA
+// visits only the key tiles listed for its query block, in ascending order;
+// every role counts its iterations the same way, so the ring and barrier
+// phases are those of a dense run over fewer tiles.
 #include "kl_common.cuh"
 #include "kl_internal.h"
 
@@ -44,6 +50,7 @@ struct AttnParams {
   const float* sv;
   uint16_t* out;
   float* amax;
+  const int* kv_list;  // nullable: per (head, query block) [count, tile indices...], n_kv + 1 ints
 };
 
 template <bool FP8>
@@ -116,13 +123,19 @@ __device__ __forceinline__ uint64_t exp2_poly_f32x2(uint64_t x2) {
   return pack_f32x2(ql, qh);
 }
 
+// entry j of a key-tile list, clamped to the tiles that exist
+__device__ __forceinline__ int tile_index(const int* list, int j, int n_kv) {
+  const int t = __ldg(list + 1 + j);
+  return t < 0 ? 0 : (t >= n_kv ? n_kv - 1 : t);
+}
+
 template <bool FP8>
 __device__ __forceinline__ void tma_tile(uint8_t* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   tma_load_2d(dst, map, x, y, bar);
   if (!FP8) tma_load_2d(dst + 16384, map, x + 64, y, bar);
 }
 
-template <bool FP8>
+template <bool FP8, bool SPARSE>
 __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const AttnParams p) {
@@ -146,7 +159,8 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qblk = blockIdx.x, h = blockIdx.y;
-  const int n = p.n_kv;
+  // dense: key tiles 0..n_kv-1; sparse: the listed ones (read after pdl_wait)
+  const int* kv_tiles = SPARSE ? p.kv_list + ((int64_t)h * gridDim.x + qblk) * (p.n_kv + 1) : nullptr;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < C::NS; ++s) {
@@ -178,6 +192,11 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   const uint32_t tmem = *tmem_holder;
   pdl_wait();  // no global memory before the previous kernel of the stream is done
   pdl_trigger();
+  int n = p.n_kv;
+  if constexpr (SPARSE) {
+    n = __ldg(kv_tiles);
+    n = n < 1 ? 1 : (n > p.n_kv ? p.n_kv : n);  // at least one tile: the last P.V signals the epilogue
+  }
   uint8_t* q_smem = smem + C::Q_OFF;
   uint8_t* kv_smem = smem + C::KV_OFF;
   uint8_t* p_smem = smem + C::P_OFF;
@@ -204,8 +223,9 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       if (elect_one()) {
         uint8_t* ks = kv_smem + s * 2 * C::TILE;
         mbar_arrive_expect_tx(&kv_full[s], 2 * C::TILE);
-        tma_tile<FP8>(ks, &tk, h * 128, j * 128, &kv_full[s]);
-        tma_tile<FP8>(ks + C::TILE, &tv, h * 128, j * 128, &kv_full[s]);
+        const int jt = SPARSE ? tile_index(kv_tiles, j, p.n_kv) : j;
+        tma_tile<FP8>(ks, &tk, h * 128, jt * 128, &kv_full[s]);
+        tma_tile<FP8>(ks + C::TILE, &tv, h * 128, jt * 128, &kv_full[s]);
       }
       __syncwarp();
       ++issued;
@@ -331,7 +351,7 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int64_t rem = p.T - (int64_t)j * 128;
+      const int64_t rem = p.T - (int64_t)(SPARSE ? tile_index(kv_tiles, j, p.n_kv) : j) * 128;
       float sc[COLS];
       float mk[8];
       // row maximum over all 128 scores: first the other half's columns
@@ -518,11 +538,13 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
   p.sv = a.sv;
   p.out = reinterpret_cast<uint16_t*>(a.out);
   p.amax = a.amax;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  p.kv_list = a.kv_list;
   const int qblocks = (int)((a.T + 128 * C::QT - 1) / (128 * C::QT));
   dim3 grid((unsigned)qblocks, (unsigned)a.H);
-  return launch_pdl(attn_kernel<FP8>, grid, dim3(C::THREADS), C::SMEM_BYTES, s, tq, tk, tv, p);
+  auto kern = a.kv_list ? attn_kernel<FP8, true> : attn_kernel<FP8, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM_BYTES, s, tq, tk, tv, p);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {

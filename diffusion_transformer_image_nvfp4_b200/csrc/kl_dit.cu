@@ -140,6 +140,7 @@ static kl_status dit_block(const DitCtx& c, int i, const uint16_t* in, uint16_t*
     b.F = c.s.F;
     b.attn_precision = c.s.attn_precision;
     b.out = y;
+    b.sol_tau = c.io->sol_tau;
     return kl_joint_block_forward(bw, &b, c.ws.block_ws, c.ws.block_ws_bytes, st);
   };
   if (i < c.s.n_mode_blocks) {  // each stream attends within itself, with its own weights

@@ -78,8 +78,16 @@ struct AttnArgs {
   int fp8;
   void* out;   // bf16 [T, H*128]
   float* amax; // nullable
+  const int* kv_list = nullptr;  // nullable: Sol-Attention key-tile lists (kl_sol_select layout)
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// Sol-Attention key-tile selection (kl_sparse.cu)
+int sol_query_rows(bool fp8);  // rows of one attention query block: 256 (FP8) / 128 (BF16)
+size_t sol_list_ints(int64_t T, int64_t H, bool fp8);
+size_t sol_workspace_bytes(int64_t T, int64_t H, bool fp8);
+cudaError_t launch_sol_select(const void* q, const void* k, int64_t ld, const float* sq, const float* sk, int64_t T,
+                              int64_t H, bool fp8, float tau, int* list, void* ws, cudaStream_t s);
 
 // tensor maps (kl_api.cu)
 // 2D tensor map, box_inner x box_outer elements; swizzle_bytes 128, 64 or 0 (none)

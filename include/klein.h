@@ -282,6 +282,45 @@ kl_status kl_joint_attention_fp8(const void* q, const void* k, const void* v, in
                                  int64_t T, int64_t H, int64_t head_dim, int precision,
                                  void* out_bf16, float* amax_out, void* stream);
 
+/*
+ * Sol-Attention ([P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA
+ * Blackwell GPUs", How it works: sparse attention leaves out less important
+ * token pairs by a sparsity threshold; What you can do: tau and a number of
+ * initial dense denoising steps).  Readings (the pages give no more): pairs
+ * are skipped one tensor-core tile at a time -- a query block (256 rows with
+ * KL_ATTN_FP8, 128 with KL_ATTN_BF16: the rows one attention CTA owns)
+ * against a key tile of 128 keys.  The estimate is
+ *   s_hat = c * (qbar . kbar),
+ * with qbar / kbar the means of the block's query rows / the tile's key rows
+ * (valid rows only at a ragged end; for KL_ATTN_FP8 the unscaled E4M3 values)
+ * and c = log2(e)/sqrt(128) (times sq[h]*sk[h] for KL_ATTN_FP8).  A tile is
+ * kept when s_hat >= max over tiles - tau (the strongest is always kept;
+ * tau = +inf keeps all).  Means and dots are fp32; the decision compares in
+ * fp32, so estimates within a few fp32 ulps of the threshold may go either way.
+ *
+ * kl_sol_select: q, k as for kl_joint_attention_fp8 (row stride ld).
+ * kv_list (device, int32, kl_sol_list_ints(T, H, precision) entries): per head
+ * h and query block b, at offset (h * n_qb + b) * (n_kt + 1) with n_qb =
+ * ceil(T / rows_per_block), n_kt = ceil(T / 128): the count, then the kept
+ * tile indices in ascending order.  workspace: >= kl_sol_workspace_size bytes,
+ * 16-byte aligned (the block means).  tau >= 0 (NaN is rejected).
+ *
+ * kl_joint_attention_sparse: kl_joint_attention_fp8 where each query block
+ * visits only the key tiles of its kv_list entry, in the given (ascending)
+ * order, with the same steps; a count outside [1, n_kt] is clamped into it
+ * and tile indices into [0, n_kt).  A list with every tile gives the dense
+ * result bit for bit.
+ */
+size_t kl_sol_list_ints(int64_t T, int64_t H, int precision);
+size_t kl_sol_workspace_size(int64_t T, int64_t H, int precision);
+kl_status kl_sol_select(const void* q, const void* k, int64_t ld, const float* scale_q, const float* scale_k,
+                        int64_t T, int64_t H, int precision, float tau, int* kv_list, void* workspace,
+                        size_t ws_bytes, void* stream);
+kl_status kl_joint_attention_sparse(const void* q, const void* k, const void* v, int64_t ld, const float* scale_q,
+                                    const float* scale_k, const float* scale_v, int64_t T, int64_t H,
+                                    int64_t head_dim, int precision, const int* kv_list, void* out,
+                                    float* amax_out, void* stream);
+
 /* ------------------------------------------------------------------------
  * The joint block
  * ---------------------------------------------------------------------- */
@@ -303,6 +342,10 @@ typedef struct kl_block_io {
                                 owned by the caller; events[i] is recorded on the
                                 stream before stage i, events[KL_BLOCK_STAGES] after
                                 the last stage (per-kernel device timing)            */
+  float sol_tau;        /* Sol-Attention threshold (log2 units): 0 (default) = dense
+                           attention; > 0 = each query block visits only the key
+                           tiles kl_sol_select keeps at this tau (selection runs
+                           inside the attention stage)                          */
 } kl_block_io;
 
 /* Stages of kl_joint_block_forward, in launch order (stage_events index). */
@@ -384,6 +427,8 @@ typedef struct kl_dit_step_io {
   const float* rope_image;
   const float* rope_joint;
   float dt;                /* t_{i+1} - t_i */
+  float sol_tau;           /* kl_block_io.sol_tau for every block of the step (0: dense;
+                              a caller keeps the first steps dense by passing 0) */
 } kl_dit_step_io;
 
 size_t kl_dit_workspace_size(const kl_dit_shape* shape);

@@ -182,3 +182,22 @@ def dit_inputs(cfg, with_weights=True, device="cpu", mods="independent"):
     else:
         raise ValueError("mods must be 'independent' or 'smooth'")
     return out
+
+
+def sparse_attention_qkv(T, H, seed, lean=8.0, spread=2.0):
+    """bf16 [T, 3*H*128] q | k | v with tile structure, for attention tile
+    skipping: per head a random unit direction u; q = N(0, 0.25) + lean * u;
+    the keys of 128-key tile j = N(0, 0.25) + a_j * u with a_j ~ U(-spread,
+    spread) (one draw per head and tile); v ~ N(0, 1).  Draw order: u, q noise,
+    a, k noise, v (torch CPU generator)."""
+    g = torch.Generator().manual_seed(seed)
+    D = H * 128
+    u = torch.randn(H, 128, generator=g, dtype=torch.float64)
+    u /= u.norm(dim=1, keepdim=True)
+    q = 0.5 * torch.randn(T, H, 128, generator=g, dtype=torch.float64) + lean * u
+    nkt = -(-T // 128)
+    a = (torch.rand(nkt, H, generator=g, dtype=torch.float64) * 2 - 1) * spread
+    a_rows = a.repeat_interleave(128, dim=0)[:T]
+    k = 0.5 * torch.randn(T, H, 128, generator=g, dtype=torch.float64) + a_rows[:, :, None] * u
+    v = torch.randn(T, H, 128, generator=g, dtype=torch.float64)
+    return torch.cat([q.reshape(T, D), k.reshape(T, D), v.reshape(T, D)], dim=1).to(torch.bfloat16)

@@ -134,3 +134,24 @@ def test_dit_cache_size_and_cached_step_validation(L):
     assert step(none, fake, need) == 2         # no block to probe
     assert L.kl_dit_cache_reset(None, None) == 1
     assert L.kl_dit_cache_reset(fake + 8, None) == 3
+
+
+def test_sol_sizes_and_validation(L):
+    T, H = 4608, 24
+    nqb8, nqb16, nkt = 18, 36, 36
+    assert L.kl_sol_list_ints(T, H, 0) == H * nqb8 * (nkt + 1)      # FP8: 256-row query blocks
+    assert L.kl_sol_list_ints(T, H, 1) == H * nqb16 * (nkt + 1)     # BF16: 128-row query blocks
+    assert L.kl_sol_workspace_size(T, H, 0) == H * (nqb8 + nkt) * 128 * 4
+    assert L.kl_sol_list_ints(0, H, 0) == 0 and L.kl_sol_workspace_size(T, H, 7) == 0
+    fake = 1 << 20
+    ws = L.kl_sol_workspace_size(T, H, 0)
+    sel = lambda tau, lst=fake, wsb=ws, sq=fake: L.kl_sol_select(fake, fake, 3 * H * 128, sq, sq, T, H, 0, tau, lst,
+                                                                 fake, wsb, None)
+    assert sel(float("nan")) == 1 and sel(-1.0) == 1           # tau must be >= 0
+    assert sel(1.0, sq=None) == 1                                # FP8 needs scales
+    assert sel(1.0, lst=None) == 1
+    assert sel(1.0, wsb=ws - 1) == 4
+    assert sel(1.0, lst=fake + 2) == 3
+    att = lambda lst, hd=128: L.kl_joint_attention_sparse(fake, fake, fake, 3 * H * 128, fake, fake, fake, T, H, hd, 0,
+                                                          lst, fake, None, None)
+    assert att(None) == 1 and att(fake, hd=64) == 2 and att(fake + 1) == 3
