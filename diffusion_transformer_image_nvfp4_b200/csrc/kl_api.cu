@@ -335,10 +335,11 @@ kl_status kl_sol_select(const void* q, const void* k, int64_t ld, const float* s
   if (precision != KL_ATTN_FP8 && precision != KL_ATTN_BF16) return KL_ERR_INVALID_ARG;
   if (precision == KL_ATTN_FP8 && (!sq || !sk)) return KL_ERR_INVALID_ARG;
   if (!(tau >= 0.f)) return KL_ERR_INVALID_ARG;  // also rejects NaN
-  if (T < 1 || H < 1 || H > 65535 || ld < H * 128 || (T + 127) / 128 > 48 * 1024) return KL_ERR_UNSUPPORTED_SHAPE;
+  if (T < 1 || H < 1 || H > 65535 || ld < H * 128 || ld % 64 || (T + 127) / 128 > 48 * 1024)
+    return KL_ERR_UNSUPPORTED_SHAPE;
   const bool fp8 = precision == KL_ATTN_FP8;
   if (!workspace || ws_bytes < sol_workspace_bytes(T, H, fp8)) return KL_ERR_WORKSPACE;
-  if (!aligned(kv_list, 4) || !aligned(workspace, 16)) return KL_ERR_MISALIGNED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(kv_list, 4) || !aligned(workspace, 16)) return KL_ERR_MISALIGNED;
   kl_status st = check_arch();
   if (st != KL_OK) return st;
   cudaError_t e = launch_sol_select(q, k, ld, sq, sk, T, H, fp8, tau, kv_list, workspace,

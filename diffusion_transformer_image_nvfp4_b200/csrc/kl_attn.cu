@@ -214,7 +214,10 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     __syncwarp();
     int issued = 0;
     bool ok = true;
+    int jt_next = SPARSE ? tile_index(kv_tiles, 0, p.n_kv) : 0;  // list entries are read one tile ahead
     for (int j = 0; j < n; ++j) {
+      const int jt = SPARSE ? jt_next : j;
+      if (SPARSE && j + 1 < n) jt_next = tile_index(kv_tiles, j + 1, p.n_kv);
       const int s = j % C::NS;
       if (!warp_wait(&kv_empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, abort_flag)) {
         ok = false;
@@ -223,7 +226,6 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       if (elect_one()) {
         uint8_t* ks = kv_smem + s * 2 * C::TILE;
         mbar_arrive_expect_tx(&kv_full[s], 2 * C::TILE);
-        const int jt = SPARSE ? tile_index(kv_tiles, j, p.n_kv) : j;
         tma_tile<FP8>(ks, &tk, h * 128, jt * 128, &kv_full[s]);
         tma_tile<FP8>(ks + C::TILE, &tv, h * 128, jt * 128, &kv_full[s]);
       }
@@ -345,13 +347,16 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
       }
     }
 #endif
+    int jt_next = SPARSE ? tile_index(kv_tiles, 0, p.n_kv) : 0;  // list entries are read one tile ahead
     for (int j = 0; j < n; ++j) {
+      const int jt = SPARSE ? jt_next : j;
+      if (SPARSE && j + 1 < n) jt_next = tile_index(kv_tiles, j + 1, p.n_kv);
       if (!warp_wait(&s_full[t], (uint32_t)j & 1u, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int64_t rem = p.T - (int64_t)(SPARSE ? tile_index(kv_tiles, j, p.n_kv) : j) * 128;
+      const int64_t rem = p.T - (int64_t)jt * 128;
       float sc[COLS];
       float mk[8];
       // row maximum over all 128 scores: first the other half's columns

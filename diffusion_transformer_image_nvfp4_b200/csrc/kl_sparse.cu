@@ -17,37 +17,63 @@
 
 namespace kl {
 
-// block means: CTA (block b, head h), thread = head dimension d; blocks
-// [0, nqb) pool query rows (q_rows each), [nqb, nqb + nkt) key rows (128 each),
-// the last of each over its valid rows only
+// block means: CTA (block b, head h), 8 warps; warp w takes rows r0 + w,
+// r0 + w + 8, ... and lane l dimensions 4l..4l+3 (a warp reads one 128-byte
+// FP8 / 256-byte BF16 row segment per step); the warps' partial sums are added
+// in warp order in shared memory.  Blocks [0, nqb) pool query rows (q_rows
+// each), [nqb, nqb + nkt) key rows (128 each), the last of each over its valid
+// rows only.
 template <bool FP8>
-__global__ void __launch_bounds__(128) sol_pool_kernel(const void* __restrict__ q, const void* __restrict__ k,
+__global__ void __launch_bounds__(256) sol_pool_kernel(const void* __restrict__ q, const void* __restrict__ k,
                                                        int64_t ld, int64_t T, int q_rows, int nqb, int nkt,
                                                        float* __restrict__ qbar, float* __restrict__ kbar) {
   pdl_wait();
   pdl_trigger();
-  const int h = blockIdx.y, d = threadIdx.x;
+  __shared__ float part[8][128];
+  const int h = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool is_q = (int)blockIdx.x < nqb;
   const int b = is_q ? blockIdx.x : blockIdx.x - nqb;
   const int rows = is_q ? q_rows : 128;
   const int64_t r0 = (int64_t)b * rows;
   const int64_t r1 = r0 + rows < T ? r0 + rows : T;
-  const int64_t col = (int64_t)h * 128 + d;
-  float acc = 0.f;
+  const int64_t col = (int64_t)h * 128 + 4 * lane;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   if (FP8) {
     const uint8_t* x = reinterpret_cast<const uint8_t*>(is_q ? q : k);
-#pragma unroll 8
-    for (int64_t r = r0; r < r1; ++r) acc += e4m3_to_f32(x[r * ld + col]);
+#pragma unroll 4
+    for (int64_t r = r0 + warp; r < r1; r += 8) {
+      const uint32_t w4 = *reinterpret_cast<const uint32_t*>(x + r * ld + col);
+      a0 += e4m3_to_f32(w4);
+      a1 += e4m3_to_f32(w4 >> 8);
+      a2 += e4m3_to_f32(w4 >> 16);
+      a3 += e4m3_to_f32(w4 >> 24);
+    }
   } else {
     const uint16_t* x = reinterpret_cast<const uint16_t*>(is_q ? q : k);
-#pragma unroll 8
-    for (int64_t r = r0; r < r1; ++r) acc += bf16_bits_to_f32(x[r * ld + col]);
+#pragma unroll 4
+    for (int64_t r = r0 + warp; r < r1; r += 8) {
+      const uint2 w4 = *reinterpret_cast<const uint2*>(x + r * ld + col);
+      a0 += bf16lo_f32(w4.x);
+      a1 += bf16hi_f32(w4.x);
+      a2 += bf16lo_f32(w4.y);
+      a3 += bf16hi_f32(w4.y);
+    }
   }
-  const float mean = acc / (float)(r1 - r0);
-  if (is_q)
-    qbar[((int64_t)h * nqb + b) * 128 + d] = mean;
-  else
-    kbar[((int64_t)h * nkt + b) * 128 + d] = mean;
+  part[warp][4 * lane] = a0;
+  part[warp][4 * lane + 1] = a1;
+  part[warp][4 * lane + 2] = a2;
+  part[warp][4 * lane + 3] = a3;
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += part[w][threadIdx.x];
+    const float mean = acc / (float)(r1 - r0);
+    if (is_q)
+      qbar[((int64_t)h * nqb + b) * 128 + threadIdx.x] = mean;
+    else
+      kbar[((int64_t)h * nkt + b) * 128 + threadIdx.x] = mean;
+  }
 }
 
 // CTA (query block b, head h), 8 warps: s_hat for every key tile (a warp per
@@ -115,9 +141,9 @@ cudaError_t launch_sol_select(const void* q, const void* k, int64_t ld, const fl
   float* qbar = reinterpret_cast<float*>(ws);
   float* kbar = qbar + (int64_t)H * nqb * 128;
   const dim3 pool_grid((unsigned)(nqb + nkt), (unsigned)H);
-  cudaError_t e = fp8 ? launch_pdl(sol_pool_kernel<true>, pool_grid, dim3(128), 0, s, q, k, ld, T, qr, nqb, nkt, qbar,
+  cudaError_t e = fp8 ? launch_pdl(sol_pool_kernel<true>, pool_grid, dim3(256), 0, s, q, k, ld, T, qr, nqb, nkt, qbar,
                                    kbar)
-                      : launch_pdl(sol_pool_kernel<false>, pool_grid, dim3(128), 0, s, q, k, ld, T, qr, nqb, nkt,
+                      : launch_pdl(sol_pool_kernel<false>, pool_grid, dim3(256), 0, s, q, k, ld, T, qr, nqb, nkt,
                                    qbar, kbar);
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)nkt * sizeof(float);

@@ -298,7 +298,8 @@ kl_status kl_joint_attention_fp8(const void* q, const void* k, const void* v, in
  * tau = +inf keeps all).  Means and dots are fp32; the decision compares in
  * fp32, so estimates within a few fp32 ulps of the threshold may go either way.
  *
- * kl_sol_select: q, k as for kl_joint_attention_fp8 (row stride ld).
+ * kl_sol_select: q, k as for kl_joint_attention_fp8 (row stride ld, a
+ * multiple of 64; q and k 16-byte aligned).
  * kv_list (device, int32, kl_sol_list_ints(T, H, precision) entries): per head
  * h and query block b, at offset (h * n_qb + b) * (n_kt + 1) with n_qb =
  * ceil(T / rows_per_block), n_kt = ceil(T / 128): the count, then the kept

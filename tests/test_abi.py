@@ -152,6 +152,8 @@ def test_sol_sizes_and_validation(L):
     assert sel(1.0, lst=None) == 1
     assert sel(1.0, wsb=ws - 1) == 4
     assert sel(1.0, lst=fake + 2) == 3
+    assert L.kl_sol_select(fake + 1, fake, 3 * H * 128, fake, fake, T, H, 0, 1.0, fake, fake, ws, None) == 3
+    assert L.kl_sol_select(fake, fake, 3 * H * 128 + 4, fake, fake, T, H, 0, 1.0, fake, fake, ws, None) == 2
     att = lambda lst, hd=128: L.kl_joint_attention_sparse(fake, fake, fake, 3 * H * 128, fake, fake, fake, T, H, hd, 0,
                                                           lst, fake, None, None)
     assert att(None) == 1 and att(fake, hd=64) == 2 and att(fake + 1) == 3
