@@ -611,42 +611,57 @@ def run_sol(args):
     scales = dict(sq=sc[:H], sk=sc[H:2 * H], sv=sc[2 * H:])
     out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    lst = kl.sol_select(q, k, T, H, 3 * D, args.sol, "fp8", sq=scales["sq"], sk=scales["sk"])
+    ws_sol = torch.empty(kl.lib().kl_sol_workspace_size(T, H, kl.ATTN["fp8"]), dtype=torch.uint8, device=dev)
 
-    def sparse_step():
-        lst = kl.sol_select(q, k, T, H, 3 * D, args.sol, "fp8", sq=scales["sq"], sk=scales["sk"])
+    def select_step():
+        kl._check(kl.lib().kl_sol_select(q.data_ptr(), k.data_ptr(), 3 * D, scales["sq"].data_ptr(),
+                                         scales["sk"].data_ptr(), T, H, kl.ATTN["fp8"], float(args.sol),
+                                         lst.data_ptr(), ws_sol.data_ptr(), ws_sol.numel(), kl._stream()),
+                  "kl_sol_select")
+
+    def sparse_step():  # selection into the preallocated list, then attention over it
+        select_step()
         kl.joint_attention_sparse(q, k, v, T, H, 3 * D, lst, "fp8", out=out, **scales)
-        return lst
 
     def dense_step():
         kl.joint_attention(q, k, v, T, H, 3 * D, "fp8", out=out, **scales)
 
     def timed(fn):
-        for _ in range(args.warmup):
+        # device time of one graph replay (no host launch gaps inside the events)
+        fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
             fn()
+        for _ in range(args.warmup):
+            graph.replay()
         ms = []
         for _ in range(args.steps):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fn()
+            graph.replay()
             b.record()
             ms.append((a, b))
         torch.cuda.synchronize()
         return statistics.median([a.elapsed_time(b) for a, b in ms])
 
-    lst = sparse_step()
+    sparse_step()
     torch.cuda.synchronize()
     nkt = -(-T // 128)
     kept = float(lst[:, :, 0].float().mean().item()) / nkt
-    t_sparse, t_dense = timed(sparse_step), timed(dense_step)
+    t_sparse, t_dense, t_select = timed(sparse_step), timed(dense_step), timed(select_step)
     flops_dense = 4.0 * T * T * H * 128
     print(json.dumps({"metric": "Sol-Attention device time (selection + sparse FP8 attention), 1024^2 T2I shape",
                       "value": round(t_sparse * 1000, 1), "unit": "us", "higher_is_better": False,
                       "dense_us": round(t_dense * 1000, 1), "speedup": round(t_dense / t_sparse, 3),
+                      "selection_us": round(t_select * 1000, 1),
                       "kept_tile_fraction": round(kept, 4), "tau": args.sol,
                       "kept_work_tflops": round(flops_dense * kept / (t_sparse * 1e-3) / 1e12, 1),
                       "config": {"workload": "sol_attention_t2i_1024", "tokens": T, "heads": H, "query_block": 256,
                                  "key_tile": 128, "inputs": "synth.sparse_attention_qkv(seed 5)",
+                                 "launch": "each leg captured in a CUDA graph, replayed per step",
                                  "l2": "flushed between timed steps (256 MiB write, outside the timed events)"},
                       "steps": args.steps, "warmup": args.warmup, "device_status": kl.device_status()}), flush=True)
 

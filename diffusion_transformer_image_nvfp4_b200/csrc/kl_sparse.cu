@@ -17,16 +17,22 @@
 
 namespace kl {
 
-// block means: CTA (block b, head h), 8 warps; warp w takes rows r0 + w,
-// r0 + w + 8, ... and lane l dimensions 4l..4l+3 (a warp reads one 128-byte
-// FP8 / 256-byte BF16 row segment per step); the warps' partial sums are added
-// in warp order in shared memory.  Blocks [0, nqb) pool query rows (q_rows
-// each), [nqb, nqb + nkt) key rows (128 each), the last of each over its valid
-// rows only.
+// block means: CTA (block b, head h), 8 warps.  A lane loads 16 bytes (16
+// E4M3 / 8 BF16 dimensions) of one row, so one warp load covers 4 (FP8) / 2
+// (BF16) rows of the head's 128 columns; warp w takes row groups w, w + 8, ...
+// with all of its loads in flight together (a query block is 8 groups per
+// warp).  Lanes holding the same dimensions are summed by shuffles, then the
+// warps' partial sums in warp order in shared memory.  Blocks [0, nqb) pool
+// query rows (q_rows each), [nqb, nqb + nkt) key rows (128 each), the last of
+// each over its valid rows only.
 template <bool FP8>
 __global__ void __launch_bounds__(256) sol_pool_kernel(const void* __restrict__ q, const void* __restrict__ k,
                                                        int64_t ld, int64_t T, int q_rows, int nqb, int nkt,
                                                        float* __restrict__ qbar, float* __restrict__ kbar) {
+  constexpr int ELEM = FP8 ? 1 : 2;
+  constexpr int DPL = 16 / ELEM;          // dimensions per lane
+  constexpr int LPR = 128 / DPL;          // lanes per row
+  constexpr int RPG = 32 / LPR;           // rows per warp load
   pdl_wait();
   pdl_trigger();
   __shared__ float part[8][128];
@@ -36,39 +42,48 @@ __global__ void __launch_bounds__(256) sol_pool_kernel(const void* __restrict__ 
   const int rows = is_q ? q_rows : 128;
   const int64_t r0 = (int64_t)b * rows;
   const int64_t r1 = r0 + rows < T ? r0 + rows : T;
-  const int64_t col = (int64_t)h * 128 + 4 * lane;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  if (FP8) {
-    const uint8_t* x = reinterpret_cast<const uint8_t*>(is_q ? q : k);
-#pragma unroll 4
-    for (int64_t r = r0 + warp; r < r1; r += 8) {
-      const uint32_t w4 = *reinterpret_cast<const uint32_t*>(x + r * ld + col);
-      a0 += e4m3_to_f32(w4);
-      a1 += e4m3_to_f32(w4 >> 8);
-      a2 += e4m3_to_f32(w4 >> 16);
-      a3 += e4m3_to_f32(w4 >> 24);
+  const int sub = lane / LPR, dim0 = (lane % LPR) * DPL;
+  const uint8_t* x = reinterpret_cast<const uint8_t*>(is_q ? q : k) + ((int64_t)h * 128 + dim0) * ELEM;
+  float acc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+  const int groups = (rows + RPG - 1) / RPG;
+  for (int g0 = 0; g0 < groups; g0 += 64) {  // one pass covers a whole block here (<= 64 groups)
+    uint4 buf[8];  // all eight loads first, then the sums (zeros past the end add nothing)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int g = g0 + warp + 8 * i;
+      const int64_t r = r0 + (int64_t)g * RPG + sub;
+      buf[i] = (g < groups && r < r1) ? *reinterpret_cast<const uint4*>(x + r * ld * ELEM) : make_uint4(0, 0, 0, 0);
     }
-  } else {
-    const uint16_t* x = reinterpret_cast<const uint16_t*>(is_q ? q : k);
-#pragma unroll 4
-    for (int64_t r = r0 + warp; r < r1; r += 8) {
-      const uint2 w4 = *reinterpret_cast<const uint2*>(x + r * ld + col);
-      a0 += bf16lo_f32(w4.x);
-      a1 += bf16hi_f32(w4.x);
-      a2 += bf16lo_f32(w4.y);
-      a3 += bf16hi_f32(w4.y);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t ww[4] = {buf[i].x, buf[i].y, buf[i].z, buf[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (FP8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[4 * j + e] += e4m3_to_f32(ww[j] >> (8 * e));
+        } else {
+          acc[2 * j] += bf16lo_f32(ww[j]);
+          acc[2 * j + 1] += bf16hi_f32(ww[j]);
+        }
+      }
     }
   }
-  part[warp][4 * lane] = a0;
-  part[warp][4 * lane + 1] = a1;
-  part[warp][4 * lane + 2] = a2;
-  part[warp][4 * lane + 3] = a3;
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  if (sub == 0)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) part[warp][dim0 + i] = acc[i];
   __syncthreads();
   if (threadIdx.x < 128) {
-    float acc = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) acc += part[w][threadIdx.x];
-    const float mean = acc / (float)(r1 - r0);
+    for (int w = 0; w < 8; ++w) sum += part[w][threadIdx.x];
+    const float mean = sum / (float)(r1 - r0);
     if (is_q)
       qbar[((int64_t)h * nqb + b) * 128 + threadIdx.x] = mean;
     else
