@@ -27,7 +27,7 @@ KL_OK = 0
 STATUS = {0: "KL_OK", 1: "KL_ERR_INVALID_ARG", 2: "KL_ERR_UNSUPPORTED_SHAPE", 3: "KL_ERR_MISALIGNED",
           4: "KL_ERR_WORKSPACE", 5: "KL_ERR_CUDA", 6: "KL_ERR_DEVICE_TIMEOUT", 7: "KL_ERR_ARCH",
           8: "KL_ERR_NONFINITE"}
-KL_SCALE_LINEAR, KL_SCALE_MMA, KL_GLOBAL_SCALE_GIVEN, KL_ROWS_SWIGLU_INTERLEAVE = 0, 1, 2, 4
+KL_SCALE_LINEAR, KL_SCALE_MMA, KL_GLOBAL_SCALE_GIVEN, KL_ROWS_SWIGLU_INTERLEAVE, KL_AMAX_GIVEN = 0, 1, 2, 4, 8
 EPI = {"none": 0, "qkv_rope": 1, "swiglu": 2, "gated_residual": 3}
 KL_OUT_BF16, KL_OUT_F32 = 0, 1
 ATTN = {"fp8": 0, "bf16": 1}
@@ -103,6 +103,8 @@ _SIGS = {
     "kl_quantize_workspace_size": ([], _SZ),
     "kl_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _I, _VP, _SZ, _VP], _I),
     "kl_ln_workspace_size": ([_I64], _SZ),
+    "kl_amax_bf16": ([_VP, _I64, _VP, _VP], _I),
+    "kl_ln_modulate_bf16": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "kl_ln_modulate_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "kl_ln_modulate_quantize_nvfp4_static": ([_VP, _I64, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP], _I),
     "kl_gemm_nvfp4_fused": ([ctypes.POINTER(_NVFP4Tensor), ctypes.POINTER(_NVFP4Tensor), _I64, _I64, _I64,
@@ -191,14 +193,31 @@ class NVFP4:
         return _NVFP4Tensor(self.codes.data_ptr(), self.scales.data_ptr(), self.gs.data_ptr())
 
 
-def quantize_nvfp4(x, layout="mma", global_scale=None, swiglu_interleave=False):
-    """kl_quantize_nvfp4 on a contiguous CUDA bf16 [R, C] tensor."""
+def quantize_nvfp4(x, layout="mma", global_scale=None, swiglu_interleave=False, amax_slot=None, out=None):
+    """kl_quantize_nvfp4 on a contiguous CUDA bf16 [R, C] tensor.  ``amax_slot``
+    (optional): a CUDA fp32 tensor of >= 64 elements, 16-byte aligned, whose
+    first element holds the tensor's amax (KL_AMAX_GIVEN: e.g. a max reduced
+    over ranks).  ``out`` (optional): an NVFP4 whose buffers are reused."""
     _need(x, torch.bfloat16, "x")
     R, C = x.shape
     L = lib()
     flags = KL_SCALE_MMA if layout == "mma" else KL_SCALE_LINEAR
+    if out is not None:
+        codes, scales, gs = out.codes, out.scales, out.gs
+        if global_scale is not None or amax_slot is None:
+            raise ValueError("out= is for the amax_slot form")
+        flags |= KL_AMAX_GIVEN
+        _check(L.kl_quantize_nvfp4(x.data_ptr(), R, C, codes.data_ptr(), scales.data_ptr(), gs.data_ptr(), flags,
+                                   amax_slot.data_ptr(), amax_slot.numel() * 4, _stream()), "kl_quantize_nvfp4")
+        return out
     codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
     scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, flags & 1), dtype=torch.uint8, device=x.device)
+    if amax_slot is not None:
+        flags |= KL_AMAX_GIVEN
+        gs = torch.empty(1, dtype=torch.float32, device=x.device)
+        _check(L.kl_quantize_nvfp4(x.data_ptr(), R, C, codes.data_ptr(), scales.data_ptr(), gs.data_ptr(), flags,
+                                   amax_slot.data_ptr(), amax_slot.numel() * 4, _stream()), "kl_quantize_nvfp4")
+        return NVFP4(codes, scales, gs, R, C, layout)
     if global_scale is not None:
         flags |= KL_GLOBAL_SCALE_GIVEN
         gs = torch.as_tensor(global_scale, dtype=torch.float32, device=x.device).reshape(1).clone()
@@ -230,6 +249,32 @@ def ln_modulate_quantize_nvfp4(x, shift, scale, export_m=False):
                                            _stream()), "kl_ln_modulate_quantize_nvfp4")
     q = NVFP4(codes, scales, gs, R, C, "mma")
     return (q, m) if export_m else q
+
+
+def amax_bf16(x, out=None):
+    """kl_amax_bf16: max|x| of a contiguous CUDA bf16 tensor (numel % 8 == 0)."""
+    _need(x, torch.bfloat16, "x")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().kl_amax_bf16(x.data_ptr(), x.numel(), out.data_ptr(), _stream()), "kl_amax_bf16")
+    return out
+
+
+def ln_modulate_bf16(x, shift, scale, m_out=None, amax_out=None):
+    """kl_ln_modulate_bf16: m = bf16(LN(x)(1+scale)+shift) and max|m|
+    max-accumulated into amax_out (zero-filled here when not given)."""
+    for t, n in ((x, "x"), (shift, "shift"), (scale, "scale")):
+        _need(t, torch.bfloat16, n)
+    R, C = x.shape
+    L = lib()
+    if m_out is None:
+        m_out = torch.empty_like(x)
+    if amax_out is None:
+        amax_out = torch.zeros(1, dtype=torch.float32, device=x.device)
+    ws = _workspace(L.kl_ln_workspace_size(R), x.device, "ln")
+    _check(L.kl_ln_modulate_bf16(x.data_ptr(), R, C, shift.data_ptr(), scale.data_ptr(), m_out.data_ptr(),
+                                 amax_out.data_ptr(), ws.data_ptr(), ws.numel(), _stream()), "kl_ln_modulate_bf16")
+    return m_out, amax_out
 
 
 def ln_modulate_quantize_nvfp4_static(x, shift, scale, export_m=False):

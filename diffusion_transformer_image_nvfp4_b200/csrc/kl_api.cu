@@ -156,7 +156,9 @@ size_t kl_quantize_workspace_size(void) { return 256; }
 kl_status kl_quantize_nvfp4(const void* x, int64_t rows, int64_t cols, void* codes, void* scales,
                             float* global_scale, int flags, void* workspace, size_t ws_bytes, void* stream) {
   if (!x || !codes || !scales || !global_scale) return KL_ERR_INVALID_ARG;
-  if (flags & ~(KL_SCALE_MMA | KL_GLOBAL_SCALE_GIVEN | KL_ROWS_SWIGLU_INTERLEAVE)) return KL_ERR_INVALID_ARG;
+  if (flags & ~(KL_SCALE_MMA | KL_GLOBAL_SCALE_GIVEN | KL_ROWS_SWIGLU_INTERLEAVE | KL_AMAX_GIVEN))
+    return KL_ERR_INVALID_ARG;
+  if ((flags & KL_GLOBAL_SCALE_GIVEN) && (flags & KL_AMAX_GIVEN)) return KL_ERR_INVALID_ARG;
   if (rows < 1 || cols < 16 || cols % 16) return KL_ERR_UNSUPPORTED_SHAPE;
   if ((flags & KL_SCALE_MMA) && cols % 64) return KL_ERR_UNSUPPORTED_SHAPE;
   if ((flags & KL_ROWS_SWIGLU_INTERLEAVE) && rows % 128) return KL_ERR_UNSUPPORTED_SHAPE;
@@ -169,11 +171,39 @@ kl_status kl_quantize_nvfp4(const void* x, int64_t rows, int64_t cols, void* cod
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* amax = reinterpret_cast<float*>(workspace);
   cudaError_t e = cudaSuccess;
-  if (!given) e = launch_amax_bf16(x, rows * cols, amax, s);
+  if (!given && !(flags & KL_AMAX_GIVEN)) e = launch_amax_bf16(x, rows * cols, amax, s);
   if (e == cudaSuccess) {
     const int mode = ((flags & KL_SCALE_MMA) ? 1 : 0) | (given ? 2 : 0) | ((flags & KL_ROWS_SWIGLU_INTERLEAVE) ? 4 : 0);
     e = launch_quantize(x, rows, cols, codes, scales, global_scale, amax, mode, s);
   }
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
+kl_status kl_amax_bf16(const void* x, int64_t n, float* amax_out, void* stream) {
+  if (!x || !amax_out) return KL_ERR_INVALID_ARG;
+  if (n < 8 || n % 8) return KL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x, 16) || !aligned(amax_out, 4)) return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  cudaError_t e = launch_amax_bf16(x, n, amax_out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
+kl_status kl_ln_modulate_bf16(const void* x, int64_t rows, int64_t cols, const void* shift, const void* scale,
+                              void* m_out, float* amax_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!x || !shift || !scale || !m_out || !amax_out) return KL_ERR_INVALID_ARG;
+  const int64_t w = cols / 256;  // the row kernel's widths
+  if (rows < 1 || cols % 256 || !(w == 1 || w == 2 || w == 4 || w == 8 || w == 12 || w == 16))
+    return KL_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x, 16) || !aligned(shift, 16) || !aligned(scale, 16) || !aligned(m_out, 16) || !aligned(amax_out, 4))
+    return KL_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < kl_ln_workspace_size(rows)) return KL_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  cudaError_t e = launch_ln_modulate_m(x, rows, cols, shift, scale, m_out,
+                                       reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace) + 256),
+                                       amax_out, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KL_OK : cuda_fail(e);
 }
 

@@ -40,6 +40,8 @@ cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t col
 cudaError_t launch_ln_modulate_quantize_via_m(const void* x, int64_t rows, int64_t cols, const void* shift,
                                              const void* scale, void* codes, void* scales, float* gs_out,
                                              void* m_buf, float2* stats, float* amax, cudaStream_t s);
+cudaError_t launch_ln_modulate_m(const void* x, int64_t rows, int64_t cols, const void* shift, const void* scale,
+                                 void* m_buf, float2* stats, float* amax, cudaStream_t s);
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s);
 cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,

@@ -578,6 +578,27 @@ cudaError_t launch_ln_modulate_quantize_via_m(const void* x, int64_t rows, int64
   return launch_quantize(m_buf, rows, cols, codes, scales, gs_out, amax, 1, s);
 }
 
+// the first half of launch_ln_modulate_quantize_via_m: m (bf16) and max|m|
+// max-accumulated into amax (the caller zero-fills it)
+cudaError_t launch_ln_modulate_m(const void* x, int64_t rows, int64_t cols, const void* shift, const void* scale,
+                                 void* m_buf, float2* stats, float* amax, cudaStream_t s) {
+  if (cols % 256) return cudaErrorInvalidValue;
+  const uint16_t* xp = reinterpret_cast<const uint16_t*>(x);
+  const uint16_t* shp = reinterpret_cast<const uint16_t*>(shift);
+  const uint16_t* scp = reinterpret_cast<const uint16_t*>(scale);
+  uint16_t* mp = reinterpret_cast<uint16_t*>(m_buf);
+  const dim3 grid((unsigned)((rows + 7) / 8)), block(256);
+  switch (cols / 256) {
+    case 1: return launch_pdl(ln_stats_rows_kernel<1>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    case 2: return launch_pdl(ln_stats_rows_kernel<2>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    case 4: return launch_pdl(ln_stats_rows_kernel<4>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    case 8: return launch_pdl(ln_stats_rows_kernel<8>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    case 12: return launch_pdl(ln_stats_rows_kernel<12>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    case 16: return launch_pdl(ln_stats_rows_kernel<16>, grid, block, 0, s, xp, rows, shp, scp, stats, amax, mp);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld, const float* amax, void* out,
                             float* scales_out, cudaStream_t s) {
   if (ncols / 128 > kFp8MaxHeads) return cudaErrorInvalidValue;

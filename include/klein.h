@@ -86,6 +86,9 @@ kl_status kl_device_status(int clear);
 #define KL_SCALE_MMA 1
 #define KL_GLOBAL_SCALE_GIVEN 2    /* use *global_scale as gs instead of amax/2688 */
 #define KL_ROWS_SWIGLU_INTERLEAVE 4/* output row r reads input row perm(r), see below */
+#define KL_AMAX_GIVEN 8            /* kl_quantize_nvfp4: the workspace's first fp32 word already
+                                      holds amax_t (e.g. a max all-reduced over ranks); the amax
+                                      pass is skipped and gs = amax_t/2688 as usual */
 
 /* Bytes of the scale array for an [R, C] NVFP4 tensor in the given layout. */
 size_t kl_nvfp4_scales_bytes(int64_t rows, int64_t cols, int layout);
@@ -102,6 +105,8 @@ size_t kl_quantize_workspace_size(void);
  * code_i = e2m1_rne_satfinite(x_i * (1/S)) (all 0 if S==0).
  * Output: codes [rows, cols/2]; scales (layout from flags); *global_scale = gs
  * (device fp32; read instead of written with KL_GLOBAL_SCALE_GIVEN).
+ * KL_AMAX_GIVEN (not with KL_GLOBAL_SCALE_GIVEN): amax_t is read from the
+ *   workspace's first fp32 word instead of computed from x.
  * KL_ROWS_SWIGLU_INTERLEAVE (rows % 128 == 0): output row r holds input row
  *   (r/128)*64 + (r%128)       if r%128 < 64   (gate half, rows [0, rows/2))
  *   rows/2 + (r/128)*64 + r%64 otherwise        (up half, rows [rows/2, rows))
@@ -131,6 +136,25 @@ kl_status kl_ln_modulate_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_
                                         void* codes, void* scales, float* global_scale,
                                         void* m_out_bf16, void* workspace, size_t ws_bytes,
                                         void* stream);
+
+/*
+ * Pieces for sequence-parallel callers, whose per-tensor scales must come
+ * from a maximum over all ranks' tokens (a max all-reduce between the pieces):
+ * kl_amax_bf16 -- *amax_out = max|x| over n bf16 values (n % 8 == 0, x 16-byte
+ *   aligned); the word is overwritten.
+ * kl_ln_modulate_bf16 -- the first half of the block's LayerNorm step:
+ *   m = bf16(LN(x) * (1 + scale) + shift) as kl_ln_modulate_quantize_nvfp4
+ *   defines it, written to m_out [rows, cols], and max|m| max-accumulated into
+ *   *amax_out (caller zero-fills).  cols / 256 in {1, 2, 4, 8, 12, 16} (the
+ *   widths the block computes m this way).  Encoding m with
+ *   kl_quantize_nvfp4(KL_SCALE_MMA | KL_AMAX_GIVEN) and the global amax gives
+ *   the block's operand bit for bit.  workspace: >= kl_ln_workspace_size(rows),
+ *   256-byte aligned (row statistics).
+ */
+kl_status kl_amax_bf16(const void* x_bf16, int64_t n, float* amax_out, void* stream);
+kl_status kl_ln_modulate_bf16(const void* x_bf16, int64_t rows, int64_t cols, const void* shift_bf16,
+                              const void* scale_bf16, void* m_out_bf16, float* amax_out, void* workspace,
+                              size_t ws_bytes, void* stream);
 
 /*
  * kl_ln_modulate_quantize_nvfp4_static -- the same computation, arguments and

@@ -157,3 +157,19 @@ def test_sol_sizes_and_validation(L):
     att = lambda lst, hd=128: L.kl_joint_attention_sparse(fake, fake, fake, 3 * H * 128, fake, fake, fake, T, H, hd, 0,
                                                           lst, fake, None, None)
     assert att(None) == 1 and att(fake, hd=64) == 2 and att(fake + 1) == 3
+
+
+def test_sequence_parallel_pieces_validation(L):
+    fake = 1 << 20
+    assert L.kl_amax_bf16(None, 64, fake, None) == 1
+    assert L.kl_amax_bf16(fake, 7, fake, None) == 2          # whole 16-byte vectors only
+    assert L.kl_amax_bf16(fake + 2, 64, fake, None) == 3
+    ws = L.kl_ln_workspace_size(100)
+    ln = lambda cols, wsb=ws, m=fake: L.kl_ln_modulate_bf16(fake, 100, cols, fake, fake, m, fake, fake, wsb, None)
+    assert ln(320) == 2 and ln(1280) == 2 and ln(5120) == 2  # widths / 256 in {1, 2, 4, 8, 12, 16} only
+    assert ln(512, m=None) == 1
+    assert ln(512, wsb=ws - 1) == 4
+    # KL_AMAX_GIVEN and KL_GLOBAL_SCALE_GIVEN exclude each other
+    assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, kl.KL_AMAX_GIVEN | kl.KL_GLOBAL_SCALE_GIVEN, fake,
+                               256, None) == 1
+    assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, kl.KL_AMAX_GIVEN, None, 0, None) == 4
