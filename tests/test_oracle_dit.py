@@ -195,3 +195,18 @@ def test_smooth_modulations_are_linear_in_t_and_keep_the_other_draws():
         step = np.abs(np.diff(m, axis=0)).mean()
         fresh = np.abs(np.diff(ind[k].double().numpy(), axis=0)).mean()
         assert step < 0.2 * fresh
+
+
+def test_cache_probe_is_the_first_joint_block_without_per_mode_blocks():
+    cfg, lat, text, w, mods, shape = _tiny(with_mode=False)
+    mods = dict(mods, mode=mods["mode"][:0])
+    cache = {}
+    v0 = dit.velocity_cached(lat, text, w, mods, shape, cache, threshold=0.5)
+    np.testing.assert_array_equal(v0, dit.velocity(lat, text, w, mods, shape))
+    # the probe residual is joint block 0's: the reference equals it exactly
+    tok = dit._embed(lat, text, w, shape)
+    f = dit._block(tok, 0, w, mods, shape, "exact")
+    np.testing.assert_array_equal(cache["r_ref"], f.astype(np.float64) - tok.astype(np.float64))
+    v1 = dit.velocity_cached(lat, text, w, mods, shape, cache, threshold=0.5)
+    assert cache["hit"] and cache["diff"] == 0.0
+    np.testing.assert_array_equal(v1, v0)
