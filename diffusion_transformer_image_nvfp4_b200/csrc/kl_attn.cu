@@ -5,8 +5,8 @@
 // tokens of the concatenated sequence ([P4] "Welcome FLUX.3 Image Klein in
 // Diffusers", Two-Stage Processing; [P2] "FLUX.3 Image Klein Brings 2-Second AI
 // Image Generation to Diffusers", Summary).  FP8 Q/K/V: [P1] "Optimizing FLUX 3
-// Image Klein inference on NVIDIA Blackwell GPUs", How it works ("Quantized
-// attention uses FP8 precision for query, key, and value").
+// Image Klein inference on NVIDIA Blackwell GPUs", How it works: the quantized
+// attention takes its query, key and value in FP8.
 //
 // One CTA = QT query tiles of 128 rows of one head (FP8: QT = 2, BF16: 1):
 //  * warp 0 lane 0 -- TMA: the Q tiles once, then K and V tiles of 128 keys
