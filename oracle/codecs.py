@@ -4,8 +4,9 @@ E2M1 and E4M3 are the element and block-scale formats of NVFP4 ([P1]
 "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs", §How it
 works, names NVFP4 weights and activations; the encoding itself is the
 standard one: E2M1 elements, unsigned E4M3 block scales).  E4M3 is also the
-FP8 format of the quantised Q/K/V attention ([P1] §How it works: "FP8
-precision for query, key, and value").  bf16 is the activation storage format.
+FP8 format of the quantised Q/K/V attention ([P1] §How it works: the
+quantised attention keeps Q, K and V in FP8).  bf16 is the activation storage
+format.
 
 Every encoder here is written as "pick the nearest representable value, ties
 to the even code, saturate to the largest finite value", evaluated exactly in
