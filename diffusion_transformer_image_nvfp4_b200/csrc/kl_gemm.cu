@@ -5,8 +5,8 @@
 // and MLP down projections.
 //
 // [P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs",
-// How it works: NVFP4 weights and activations feed optimised GEMM kernels that
-// fuse SwiGLU activations and rotary position embeddings.  The page names
+// How it works: the projections run NVFP4 x NVFP4 in GEMM kernels that also
+// apply the SwiGLU gate and the rotary embedding in place.  The page names
 // those kernels (PrimsTS) but gives no design; this one is written for B200:
 //
 //  * persistent grid (one 352-thread CTA per SM), 128 x BN output tiles,

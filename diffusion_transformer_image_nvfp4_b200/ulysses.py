@@ -3,7 +3,8 @@
 [P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs", How
 it works: to use several GPUs, the token sequence is split between them
 (Ulysses) and attention is computed in a distributed way that still sees
-every token; What you can do: ``ulysses_size`` in the parallel config.
+every token; What you can do: the degree of this split is a setting
+(``ulysses_size``).
 
 The tokens of one sequence are sharded over the N ranks of a process group
 (rank r holds tokens [r T/N, (r+1) T/N)); the weights are replicated.  Every

@@ -6,11 +6,12 @@
  *
  * Sources (page titles and sections):
  *  [P1] "Optimizing FLUX 3 Image Klein inference on NVIDIA Blackwell GPUs",
- *       How it works: NVFP4 weights and activations; GEMM kernels that fuse
- *       SwiGLU and rotary position embeddings; FP8 query/key/value attention.
+ *       How it works: NVFP4 weights and activations; GEMM kernels with the
+ *       SwiGLU gate and the rotary embedding folded in; attention on FP8 Q/K/V.
  *  [P2] "FLUX.3 Image Klein Brings 2-Second AI Image Generation to Diffusers",
- *       Summary: 28 joint transformer blocks merge text, generated-image and
- *       reference tokens; a 1024x1024 reference adds 4,096 tokens.
+ *       Summary: 28 joint blocks run over one sequence of text, target-image
+ *       and reference-image tokens; each 1024x1024 reference brings another
+ *       4,096 tokens.
  *  [P4] "Welcome FLUX.3 Image Klein in Diffusers", Architecture and Technical
  *       Deep Dive: 64x64 = 4,096 tokens per 1024x1024 image; 3072-wide
  *       transformer; joint blocks attend over the concatenated streams.
