@@ -63,10 +63,7 @@ struct AttnCfg {
   static constexpr float TAU = FP8 ? 4.0f : 8.0f;  // lazy-rescale threshold, log2 units
   static constexpr float P_SCALE = FP8 ? 16.0f : 1.0f;  // p * P_SCALE <= 2^(TAU+4) <= 448
   static constexpr float LOG2_P_SCALE = FP8 ? 4.0f : 0.0f;
-#ifndef KL_ATTN_SPLIT
-#define KL_ATTN_SPLIT 2
-#endif
-  static constexpr int SPLIT = KL_ATTN_SPLIT;     // softmax warps per 32 query rows (1 or 2)
+  static constexpr int SPLIT = 2;                  // softmax warps per 32 query rows
   static constexpr int COLS = 128 / SPLIT;         // score / output columns per softmax thread
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = QT * TILE;
@@ -80,48 +77,6 @@ struct AttnCfg {
   static constexpr int SMEM_BYTES = L_OFF + QT * SPLIT * 128 * 4 + 1024;
   static_assert(SMEM_BYTES <= 232448, "smem budget");
 };
-
-// Share of the softmax exponentials computed on the FMA pipe instead of the
-// MUFU unit: KL_ATTN_POLY of every 8 element pairs.  The MUFU unit issues a
-// quarter warp of ex2 per cycle per SM sub-partition, which alone would hold
-// the softmax to about half the FP8 tensor-core rate; running some of the
-// exponentials as FMAs keeps both pipes busy.
-#ifndef KL_ATTN_STAGGER
-#define KL_ATTN_STAGGER 0
-#endif
-#ifndef KL_ATTN_POLY
-#define KL_ATTN_POLY 0
-#endif
-
-// 2^x for two floats on the FMA pipe.  Cody-Waite style range reduction
-// x = j + f, j = rint(x) (the 1.5 * 2^23 add rounds to an integer), |f| <= 1/2;
-// 2^f by a degree-4 polynomial whose coefficients were fitted here to the
-// relative error of 2^f on [-1/2, 1/2] (Lawson-weighted least squares; max
-// relative error 2.9e-6 in fp32 Horner form, far below the E4M3 rounding of
-// p that follows); 2^j is added to the exponent field (j << 23).  x is
-// clamped to >= -125 so the exponent stays normal; 2^-125 rounds to 0 in
-// E4M3 like the exact value would.
-__device__ __forceinline__ uint64_t exp2_poly_f32x2(uint64_t x2) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  float xl, xh;
-  unpack_f32x2(x2, xl, xh);
-  const uint64_t x = pack_f32x2(fmaxf(xl, -125.0f), fmaxf(xh, -125.0f));
-  const uint64_t t = add_f32x2(x, pack_f32x2(kRound, kRound));
-  const uint64_t jf = add_f32x2(t, pack_f32x2(-kRound, -kRound));
-  const uint64_t f = fma_f32x2(jf, pack_f32x2(-1.0f, -1.0f), x);
-  uint64_t q = fma_f32x2(pack_f32x2(0.009582853f, 0.009582853f), f, pack_f32x2(0.055906426f, 0.055906426f));
-  q = fma_f32x2(q, f, pack_f32x2(0.24024099f, 0.24024099f));
-  q = fma_f32x2(q, f, pack_f32x2(0.69312418f, 0.69312418f));
-  q = fma_f32x2(q, f, pack_f32x2(1.0f, 1.0f));
-  float ql, qh, tl, th;
-  unpack_f32x2(q, ql, qh);
-  unpack_f32x2(t, tl, th);
-  // bits(t) = bits(1.5 * 2^23) + j and bits(1.5 * 2^23) is a multiple of 2^9,
-  // so bits(t) << 23 == j << 23 (mod 2^32)
-  ql = __int_as_float(__float_as_int(ql) + (int)((uint32_t)__float_as_int(tl) << 23));
-  qh = __int_as_float(__float_as_int(qh) + (int)((uint32_t)__float_as_int(th) << 23));
-  return pack_f32x2(ql, qh);
-}
 
 // entry j of a key-tile list, clamped to the tiles that exist
 __device__ __forceinline__ int tile_index(const int* list, int j, int n_kv) {
@@ -340,13 +295,6 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     if (FP8) c *= __ldg(p.sq + h) * __ldg(p.sk + h);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-#if KL_ATTN_STAGGER
-    if (t == 1) {
-      const long long t0 = clock64();
-      while (clock64() - t0 < KL_ATTN_STAGGER) {
-      }
-    }
-#endif
     int jt_next = SPARSE ? tile_index(kv_tiles, 0, p.n_kv) : 0;  // list entries are read one tile ahead
     for (int j = 0; j < n; ++j) {
       const int jt = SPARSE ? jt_next : j;
@@ -427,14 +375,10 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
 #pragma unroll
       for (int i = 0; i < COLS; i += 2) {
         const uint64_t x2 = fma_f32x2(pack_f32x2(sc[i], sc[i + 1]), c2, mb2);
-        if (((i >> 1) & 7) < KL_ATTN_POLY) {
-          unpack_f32x2(exp2_poly_f32x2(x2), sc[i], sc[i + 1]);
-        } else {
-          float lo, hi;
-          unpack_f32x2(x2, lo, hi);
-          sc[i] = ex2_approx(lo);
-          sc[i + 1] = ex2_approx(hi);
-        }
+        float lo, hi;
+        unpack_f32x2(x2, lo, hi);
+        sc[i] = ex2_approx(lo);
+        sc[i + 1] = ex2_approx(hi);
         acc2[(i >> 1) & 3] = add_f32x2(acc2[(i >> 1) & 3], pack_f32x2(sc[i], sc[i + 1]));
       }
       float a0, a1, b0, b1;
