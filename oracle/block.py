@@ -202,18 +202,59 @@ def fp8_encode_heads(x):
     return e4m3_round(y), s
 
 
-def attention_fp8_emulated(q, k, v, tile=128, p_scale=16.0, tau=4.0, rows=None):
-    """FP8 joint attention as a flash-style kernel computes it (a reading; the
-    pages name FP8 Q/K/V attention but not its arithmetic).
+def fp8_flash_rows(q8, k8, v8, c, key_tiles=None, tile=128, p_scale=16.0, tau=4.0):
+    """One head's flash-style pass over E4M3 operands (a reading; see below).
 
-    Q, K and V are rounded to E4M3 after scaling each head by 448 / amax.
-    Keys are visited in tiles of ``tile``.  Per query row a reference maximum
-    m of the scaled log2 scores t = (q8 . k8) * sq * sk * log2(e) / sqrt(d) is
-    kept; it is only moved -- and the output accumulator and row sum l are
-    rescaled by 2^(m_old - m_new) -- when a tile's maximum exceeds m by more
-    than ``tau``, so every p = 2^(t - m) <= 2^tau.  p * ``p_scale`` is rounded
-    to E4M3 and multiplied with v8; l sums the unrounded p.
-    O = acc * s_v / (p_scale * l).  Everything else fp64.
+    q8 [R, d], k8 [T, d], v8 [T, d]: decoded E4M3 values (unscaled); c: the
+    factor that turns q8 . k8 into log2 units of the softmax argument;
+    key_tiles: the tiles of ``tile`` keys to visit, in order (default: all).
+    Returns (acc, l) with O = acc / (p_scale * l) times the V decode scale.
+
+    Steps, per visited tile: t = (q8 . k8) * c for its keys; the row's
+    reference maximum m (initially -inf) is moved to the tile maximum only
+    when that exceeds m by more than ``tau``, and then acc and l are first
+    multiplied by 2^(m_old - m_new); p = 2^(t - m), so p <= 2^tau;
+    acc += e4m3(p * p_scale) . v8 and l += sum of the unrounded p.  Visiting
+    keys a tile at a time with a running maximum is the flash-attention
+    scheme; moving the maximum only past a threshold is the conditional
+    rescale of the Blackwell flash-attention design (the normalisation is
+    unchanged: rescaling by any common reference gives the same softmax).
+    Its effect here is where P is rounded: with p_scale = 16 and tau = 4,
+    p * p_scale <= 256 stays inside E4M3's range (448).
+    """
+    q8 = np.asarray(q8, np.float64)
+    k8 = np.asarray(k8, np.float64)
+    v8 = np.asarray(v8, np.float64)
+    R, d = q8.shape
+    T = k8.shape[0]
+    if key_tiles is None:
+        key_tiles = range(-(-T // tile))
+    m = np.full(R, -np.inf)
+    l = np.zeros(R)
+    acc = np.zeros((R, v8.shape[1]))
+    for j in key_tiles:
+        j0 = j * tile
+        t = (q8 @ k8[j0:j0 + tile].T) * c
+        mx = t.max(axis=1)
+        move = mx > m + tau
+        alpha = np.where(move, np.exp2(np.where(move, m - mx, 0.0)), 1.0)
+        acc *= alpha[:, None]
+        l *= alpha
+        m = np.where(move, mx, m)
+        p = np.exp2(t - m[:, None])
+        l += p.sum(axis=1)
+        acc += e4m3_round(p * p_scale) @ v8[j0:j0 + tile]
+    return acc, l
+
+
+def attention_fp8_emulated(q, k, v, tile=128, p_scale=16.0, tau=4.0, rows=None):
+    """FP8 joint attention, flash-style (a reading; the pages name FP8 Q/K/V
+    attention but not its arithmetic).
+
+    Q, K and V are rounded to E4M3 after scaling each head by 448 / amax
+    (``fp8_encode_heads``); the softmax argument in log2 units is
+    t = (q8 . k8) * sq * sk * log2(e) / sqrt(d); ``fp8_flash_rows`` visits all
+    key tiles in order; O = acc * s_v / (p_scale * l).  Everything else fp64.
     ``rows`` optionally restricts the query rows (scales still use all rows).
     """
     q8, sq = fp8_encode_heads(q)
@@ -226,21 +267,7 @@ def attention_fp8_emulated(q, k, v, tile=128, p_scale=16.0, tau=4.0, rows=None):
     out = np.empty((R, H, d), dtype=np.float64)
     for h in range(H):
         c = np.log2(np.e) / np.sqrt(d) * float(sq[h]) * float(sk[h])
-        m = np.full(R, -np.inf)
-        l = np.zeros(R)
-        acc = np.zeros((R, d))
-        for j0 in range(0, T, tile):
-            t = (q8[:, h, :] @ k8[j0:j0 + tile, h, :].T) * c
-            mx = t.max(axis=1)
-            move = mx > m + tau
-            alpha = np.where(move, np.exp2(np.where(move, m - mx, 0.0)), 1.0)
-            acc *= alpha[:, None]
-            l *= alpha
-            m = np.where(move, mx, m)
-            p = np.exp2(t - m[:, None])
-            p8 = e4m3_round(p * p_scale)
-            l += p.sum(axis=1)
-            acc += p8 @ v8[j0:j0 + tile, h, :]
+        acc, l = fp8_flash_rows(q8[:, h, :], k8[:, h, :], v8[:, h, :], c, tile=tile, p_scale=p_scale, tau=tau)
         out[:, h, :] = acc * float(sv[h]) / (p_scale * l[:, None])
     return out
 

@@ -27,8 +27,7 @@ library's kl_sol_select / kl_joint_attention_sparse):
 
 import numpy as np
 
-from .block import attention, fp8_encode_heads
-from .codecs import e4m3_round
+from .block import attention, fp8_encode_heads, fp8_flash_rows
 
 LOG2E = np.log2(np.e)
 
@@ -79,10 +78,9 @@ def attention_sparse_exact(q, k, v, keep, q_block, tile=128):
 
 
 def attention_fp8_emulated_sparse(q, k, v, keep, q_block, tile=128, p_scale=16.0, tau=4.0):
-    """The FP8 kernel's steps (E4M3 Q/K/V with per-head scales over all
-    tokens, lazy rescale when a tile's maximum passes m by more than tau, P *
-    p_scale rounded to E4M3, unrounded row sums) with each query block
-    visiting only its kept key tiles, in ascending order."""
+    """The FP8 reading of ``block.attention_fp8_emulated`` (E4M3 Q/K/V with
+    per-head scales over all tokens, ``block.fp8_flash_rows``) with each query
+    block visiting only its kept key tiles, in ascending order."""
     q8, sq = fp8_encode_heads(q)
     k8, sk = fp8_encode_heads(k)
     v8, sv = fp8_encode_heads(v)
@@ -92,22 +90,8 @@ def attention_fp8_emulated_sparse(q, k, v, keep, q_block, tile=128, p_scale=16.0
         c = LOG2E / np.sqrt(d) * float(sq[h]) * float(sk[h])
         for b in range(keep.shape[1]):
             rows = np.arange(b * q_block, min((b + 1) * q_block, T))
-            R = len(rows)
-            m = np.full(R, -np.inf)
-            l = np.zeros(R)
-            acc = np.zeros((R, d))
-            for j in np.flatnonzero(keep[h, b]):
-                j0 = j * tile
-                t = (q8[rows, h, :] @ k8[j0:j0 + tile, h, :].T) * c
-                mx = t.max(axis=1)
-                move = mx > m + tau
-                alpha = np.where(move, np.exp2(np.where(move, m - mx, 0.0)), 1.0)
-                acc *= alpha[:, None]
-                l *= alpha
-                m = np.where(move, mx, m)
-                p = np.exp2(t - m[:, None])
-                l += p.sum(axis=1)
-                acc += e4m3_round(p * p_scale) @ v8[j0:j0 + tile, h, :]
+            acc, l = fp8_flash_rows(q8[rows, h, :], k8[:, h, :], v8[:, h, :], c, np.flatnonzero(keep[h, b]),
+                                    tile=tile, p_scale=p_scale, tau=tau)
             out[rows, h, :] = acc * float(sv[h]) / (p_scale * l[:, None])
     return out
 

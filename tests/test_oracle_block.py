@@ -300,7 +300,7 @@ def test_block_runs_on_tiny_workload():
 
 
 def test_fp8_emulation_uniform_scores_give_mean_of_quantised_values():
-    # q = 0 makes every score 0, every p exactly 1 (p * 256 = 256 is an E4M3
+    # q = 0 makes every score 0, every p exactly 1 (p * 16 = 16 is an E4M3
     # value), so O is the plain mean of the E4M3-decoded v, over any tiling
     rng = np.random.default_rng(12)
     T, H = 300, 2
@@ -326,3 +326,89 @@ def test_fp8_emulation_close_to_exact_and_rows_subset():
     np.testing.assert_allclose(block.attention_fp8_emulated(q, k, v, rows=rows), emu[rows], rtol=1e-13)
     s, inv = block.fp8_head_scales(v)
     np.testing.assert_allclose(s * inv, 1.0, rtol=1e-6)
+
+
+def _integer_score_case(seed, R=24, tiles=(0, 6, 9, 15, 13), tile=128, T=600):
+    """E4M3-valued q8 [R, d], k8 [T, d], v8 [T, d] whose scores q8 . k8 are
+    small integers: key j of tile i scores base_i - u_j + a_r * b_j with
+    u_j in [0, 9] (0 at the tile's first key and at its key 64, so 64-key
+    tiles have the same maxima), a_r in {-1, 0, 1}, b_j in {0, 1}.  With
+    c = 1 every p = 2^(t - m) is then a power of two; the tile maxima rise
+    by more than 4 at tiles 1 and 3, so the running maximum moves there."""
+    rng = np.random.default_rng(seed)
+    d = 128
+    s = np.empty(T)
+    for i, base in enumerate(tiles):
+        j0, j1 = i * tile, min(T, (i + 1) * tile)
+        u = rng.integers(0, 10, j1 - j0).astype(np.float64)
+        u[0] = 0.0
+        if j1 - j0 > 64:
+            u[64] = 0.0
+        s[j0:j1] = base - u
+    a = rng.integers(-1, 2, R).astype(np.float64)
+    b = rng.integers(0, 2, T).astype(np.float64)
+    q8 = np.zeros((R, d))
+    q8[:, 0] = 1.0
+    q8[:, 1] = a
+    k8 = np.zeros((T, d))
+    k8[:, 0] = s
+    k8[:, 1] = b
+    v8 = codecs.e4m3_round(rng.standard_normal((T, d)) * 8.0)
+    t = q8 @ k8.T
+    assert np.array_equal(t, np.round(t)) and np.abs(k8).max() <= 16   # integers, exact in E4M3
+    return q8, k8, v8, t
+
+
+def _softmax2(t, v8):
+    """sum_j 2^t_j v_j / sum_j 2^t_j in fp64 (the softmax in base 2)."""
+    w = np.exp2(t - t.max(axis=1, keepdims=True))
+    return (w @ v8) / w.sum(axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("tau,tile", [(4.0, 128), (0.0, 128), (4.0, 64), (0.0, 64)])
+def test_fp8_flash_rescale_is_exact_on_power_of_two_probabilities(tau, tile):
+    # Every p * 16 is a power of two in [2^-9, 256], so E4M3 holds it exactly,
+    # and the tile-by-tile pass must equal the plain softmax over the same
+    # operands up to fp64 rounding -- through every move of the running
+    # maximum (tiles 1 and 3 always move it; tau = 0 moves it whenever a tile
+    # maximum rises).  A rescale of acc or l that is dropped, applied twice or
+    # given the wrong sign breaks this by a factor of 2^5 or more.
+    q8, k8, v8, t = _integer_score_case(21)
+    acc, l = block.fp8_flash_rows(q8, k8, v8, 1.0, tile=tile, p_scale=16.0, tau=tau)
+    np.testing.assert_allclose(acc / (16.0 * l[:, None]), _softmax2(t, v8), rtol=1e-12, atol=1e-12)
+    # l itself is the sum of 2^(t - m_final), m_final the last reference maximum
+    m_final = t[:, 384:512].max(axis=1)   # set at tile 3, never moved after it
+    np.testing.assert_allclose(l, np.exp2(t - m_final[:, None]).sum(axis=1), rtol=1e-13)
+
+
+def test_fp8_flash_visits_only_the_listed_tiles_in_order():
+    # the same exact case restricted to a list of key tiles: equal to the
+    # softmax over those tiles' keys (ascending lists, as the sparse path uses)
+    q8, k8, v8, t = _integer_score_case(22)
+    for tiles in ([0, 1, 3], [1, 2, 3, 4], [0, 3, 4], [3]):
+        cols = np.concatenate([np.arange(j * 128, min(600, (j + 1) * 128)) for j in tiles])
+        acc, l = block.fp8_flash_rows(q8, k8, v8, 1.0, key_tiles=tiles)
+        np.testing.assert_allclose(acc / (16.0 * l[:, None]), _softmax2(t[:, cols], v8[cols]), rtol=1e-12,
+                                   atol=1e-12)
+
+
+def test_fp8_flash_rounds_p_for_the_product_but_sums_the_unrounded_p():
+    # Two keys whose log2 scores are 0 and log2(1.1): the tile maximum is
+    # log2(1.1), so p = (1/1.1, 1) and p * 16 = (14.545..., 16).  E4M3 has
+    # steps of 1 on [8, 16): 14.545... rounds to 15 and 16 stays.  The product
+    # uses the rounded values, the row sum the unrounded ones:
+    # O = (15 v0 + 16 v1) / (16 * (1/1.1 + 1)).
+    d = 128
+    q8 = np.zeros((1, d))
+    q8[0, 0] = 1.0
+    k8 = np.zeros((2, d))
+    k8[1, 0] = 1.0
+    v8 = np.zeros((2, d))
+    v8[0, 0] = 1.0
+    v8[1, 1] = 2.0
+    acc, l = block.fp8_flash_rows(q8, k8, v8, math.log2(1.1))
+    np.testing.assert_allclose(l, [1.0 / 1.1 + 1.0], rtol=1e-15)
+    want = np.zeros(d)
+    want[0] = 15.0 / (16.0 * (1.0 / 1.1 + 1.0))
+    want[1] = 32.0 / (16.0 * (1.0 / 1.1 + 1.0))
+    np.testing.assert_allclose(acc[0] / (16.0 * l[0]), want, rtol=1e-14, atol=1e-15)

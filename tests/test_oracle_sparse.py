@@ -84,3 +84,28 @@ def test_a_far_away_tile_is_skipped_without_changing_the_output():
     q8, k8, c8 = sparse.fp8_select_inputs(q, k)
     keep8, _ = sparse.sol_select(q8, k8, c8, 4.0, 256)
     assert not keep8[0, :, 1].any()
+
+
+def test_fp8_sparse_emulation_equals_the_dense_emulation_over_the_kept_keys():
+    # When every kept list holds the tile that carries each head's largest |k|
+    # and |v| (tile 0 here), the per-head E4M3 scales over all tokens equal
+    # those over the kept keys, so each query block's sparse pass must equal
+    # the dense FP8 emulation run on just its kept keys (full 128-key tiles,
+    # so the tile boundaries coincide).  This pins the per-block bookkeeping
+    # of the sparse wrapper; the tile-by-tile steps themselves are pinned
+    # exactly in test_oracle_block.py.
+    T, H, d = 512, 2, 128
+    q, k, v = _qkv(T, H, d, 5)
+    k[3] *= 4.0
+    v[5] *= 4.0
+    keep = np.array([[[True, False, True, True], [True, True, False, False]],
+                     [[True, True, True, False], [True, False, False, True]]])
+    got = sparse.attention_fp8_emulated_sparse(q, k, v, keep, 256)
+    for h in range(H):
+        for b in range(2):
+            rows = np.arange(b * 256, (b + 1) * 256)
+            cols = sparse.kept_key_rows(keep[h, b], T)
+            qq = np.concatenate([q[rows][:, h:h + 1], q[:, h:h + 1]])   # all rows keep the q scale unchanged
+            want = block.attention_fp8_emulated(qq, k[cols][:, h:h + 1], v[cols][:, h:h + 1],
+                                                 rows=np.arange(len(rows)))
+            np.testing.assert_allclose(got[rows, h], want[:, 0], rtol=0, atol=1e-12)
