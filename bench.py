@@ -255,18 +255,39 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, n_text=256, grid_rows=4):
+def _oracle_block_seconds(wl, n_text, grid_rows):
     from oracle import block
 
     x, mod, w, lay = oracle_sample(wl, n_text, grid_rows)
     attn = "fp8" if wl.attn == "fp8" else "exact"
     t0 = time.perf_counter()
     block.block_forward(x, mod, w, lay, wl.heads, attn=attn)
-    dt = time.perf_counter() - t0
-    T = lay.n_tokens
-    return {"value": round(T / dt, 3), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{T}-token slice of {wl.name} ({n_text} text + {grid_rows} grid rows x {wl.grid_w}), "
-                      f"full widths, weights pre-encoded (untimed), one block forward: {dt:.1f} s"}
+    return time.perf_counter() - t0, lay.n_tokens
+
+
+def cpu_baseline(wl, n_text=256, grid_rows=4):
+    """The oracle on the host cores: a bounded slice of the workload with all
+    BLAS threads, plus single-thread figures (the whole tiny block, and a
+    128-token slice of this workload)."""
+    dt, T = _oracle_block_seconds(wl, n_text, grid_rows)
+    out = {"value": round(T / dt, 3), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"{T}-token slice of {wl.name} ({n_text} text + {grid_rows} grid rows x {wl.grid_w}), "
+                     f"full widths, weights pre-encoded (untimed), one block forward: {dt:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return out
+    single = {}
+    with threadpool_limits(limits=1):
+        tiny = WORKLOADS["tiny"]
+        dt1, T1 = _oracle_block_seconds(tiny, tiny.n_text, tiny.grid_h)
+        single["tiny"] = {"value": round(T1 / dt1, 3), "unit": UNIT, "cores": 1,
+                          "sample": f"the whole tiny block ({T1} tokens): {dt1:.1f} s"}
+        dt2, T2 = _oracle_block_seconds(wl, 64, 1)
+        single[wl.name] = {"value": round(T2 / dt2, 3), "unit": UNIT, "cores": 1,
+                           "sample": f"{T2}-token slice of {wl.name} (64 text + 1 grid row), full widths: {dt2:.1f} s"}
+    out["single_thread"] = single
+    return out
 
 
 def run_reference(args, wl):
@@ -302,9 +323,21 @@ def run_reference(args, wl):
 
 
 # ------------------------------------------------------------------------ ours
-def secondary_block(kl, wl, dev, steps, warmup, flush, world):
-    """Graph-replay tokens/s of another workload's block (same method as the
-    main measurement, L2 flushed before every step, max over ranks)."""
+GATE_CYCLES = 20_000_000   # ~10 ms at B200 clocks: covers enqueueing a chunk of steps
+CHUNK = 16
+
+
+def gated(n_steps, body):
+    """Enqueue the steps in chunks behind a short GPU sleep, so the queue is
+    already full when the GPU reaches them and host-side enqueue time never
+    shows up as device time."""
+    for c0 in range(0, n_steps, CHUNK):
+        torch.cuda._sleep(GATE_CYCLES)
+        for i in range(c0, min(n_steps, c0 + CHUNK)):
+            body(i)
+
+
+def block_setup(kl, wl, dev):
     inp = block_inputs(wl)
     T, D, H, F = wl.n_tokens, wl.hidden, wl.heads, wl.mlp_hidden
     d = {k: v.to(dev) for k, v in inp.items()}
@@ -313,29 +346,130 @@ def secondary_block(kl, wl, dev, steps, warmup, flush, world):
     mod = {n: d[n] for n in MOD_NAMES}
     out = torch.empty_like(d["x"])
     ws = torch.empty(kl.block_workspace_size(T, D, H, F, wl.attn), dtype=torch.uint8, device=dev)
+    return inp, W, cs, d["x"], mod, out, ws
+
+
+def measure_block(kl, wl, dev, steps, warmup, flush, world, peaks, clocks=None, e2e=False):
+    """One workload's block: graph-replay tokens/s (L2 flushed before every
+    step), per-stage device times from direct launches with library-recorded
+    events, roofline fractions; with ``e2e`` also the end-to-end number
+    through kl_joint_block_forward_host on pinned host buffers."""
+    inp, W, cs, x, mod, out, ws = block_setup(kl, wl, dev)
+    T, D, H, F = wl.n_tokens, wl.hidden, wl.heads, wl.mlp_hidden
     for _ in range(warmup):
-        kl.joint_block_forward(W, d["x"], mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
+        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    st = kl.device_status()
+    if st != "KL_OK":
+        raise SystemExit(f"{wl.name}: device status after warm-up: {st}")
+
+    # value: the block captured once in a CUDA graph and replayed; every step
+    # an L2 flush, then one replay bracketed by events on the stream
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        kl.joint_block_forward(W, d["x"], mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
+        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
     for _ in range(3):
         graph.replay()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    rank_barrier(world, dev)
-    torch.cuda._sleep(20_000_000)
-    for a, b in ev:
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+
+    def graph_step(i):
         flush.zero_()
-        a.record()
+        starts[i].record()
         graph.replay()
-        b.record()
+        ends[i].record()
+
     rank_barrier(world, dev)
-    total_ms = rank_max(sum(a.elapsed_time(b) for a, b in ev), world, dev)
+    if clocks is not None:
+        clocks.start()
+    gated(steps, graph_step)
+    rank_barrier(world, dev)
+    clk = clocks.stop() if clocks is not None else None
+    total_ms = rank_max(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, dev)
     del graph
+
+    # per-stage breakdown: the same steps launched directly, the library
+    # recording an event between the stages of every step
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(steps)]
+    for row in stage_ev:
+        for e in row:
+            e.record()
+
+    def eager_step(i):
+        flush.zero_()
+        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws, stage_events=stage_ev[i])
+
+    rank_barrier(world, dev)
+    gated(steps, eager_step)
+    rank_barrier(world, dev)
+    stage_ms = {s: sum(row[j].elapsed_time(row[j + 1]) for row in stage_ev) / steps for j, s in enumerate(STAGES)}
+    eager_ms = sum(row[0].elapsed_time(row[-1]) for row in stage_ev) / steps
+
+    res = {"workload": wl.name, "tokens": T, "steps": steps, "total_ms": total_ms, "clk": clk,
+           "stage_ms": stage_ms, "eager_ms": eager_ms}
+    if e2e:
+        # end to end through the C ABI with host buffers: every step one
+        # kl_joint_block_forward_host call (pinned x and modulation copied in,
+        # the block, out copied back), all inside the timed events
+        x_h = inp["x"].pin_memory()
+        mod_h = {n: inp[n].pin_memory() for n in MOD_NAMES}
+        out_h = torch.empty_like(x_h).pin_memory()
+        ws_h = torch.empty(kl.lib().kl_block_host_workspace_size(T, D, H, F, kl.ATTN[wl.attn]), dtype=torch.uint8,
+                           device=dev)
+        kl.joint_block_forward_host(W, x_h, mod_h, cs, H, F, attn=wl.attn, out_host=out_h, workspace=ws_h)
+        torch.cuda.synchronize()
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+
+        def e2e_step(i):
+            flush.zero_()
+            e2e_ev[i][0].record()
+            kl.joint_block_forward_host(W, x_h, mod_h, cs, H, F, attn=wl.attn, out_host=out_h, workspace=ws_h)
+            e2e_ev[i][1].record()
+
+        rank_barrier(world, dev)
+        gated(steps, e2e_step)
+        rank_barrier(world, dev)
+        res["e2e_ms"] = rank_max(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev)
+        res["h2d"] = T * D * 2 + len(MOD_NAMES) * D * 2
+        res["d2h"] = T * D * 2
+        if not torch.equal(out_h.to(dev), out):
+            raise SystemExit(f"{wl.name}: host-buffer entry point disagrees with the device one")
+    st = kl.device_status()
+    if st != "KL_OK":
+        raise SystemExit(f"{wl.name}: device status after timing: {st}")
+    return res
+
+
+def summarize(wl, res, peaks, pk, world):
+    """tokens/s, TFLOP/s, per-stage roofline entries and the GEMM / attention
+    fractions of one measured workload."""
+    steps, total_ms, stage_ms = res["steps"], res["total_ms"], res["stage_ms"]
     work = stage_work(wl)
-    gemm_flop = sum(work[s][1] for s in ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm"))
-    return {"workload": wl.name, "tokens": T, "value": round(whole_job_value(world, T, steps, total_ms), 1),
-            "unit": UNIT, "ms_per_step": round(total_ms / steps, 4), "steps": steps,
-            "tflops": round((gemm_flop + work["attention"][1]) / (total_ms / steps * 1e-3) / 1e12, 2)}
+    stages = {}
+    for s in STAGES:
+        if wl.attn != "fp8" and s == "fp8_cast":
+            continue
+        ent = roofline_entry(work[s], stage_ms[s], peaks, pk) or {}
+        ent["ms"] = round(stage_ms[s], 4)
+        stages[s] = ent
+    gemms = ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm")
+    gemm_ms = sum(stage_ms[s] for s in gemms)
+    gemm_flop = sum(work[s][1] for s in gemms)
+    fp4_peak = peaks[pk] * RATIO["fp4"]
+    att_peak = peaks[pk] * RATIO["fp8" if wl.attn == "fp8" else "bf16"]
+    return {"workload": wl.name, "tokens": wl.n_tokens,
+            "value": round(whole_job_value(world, wl.n_tokens, steps, total_ms), 1), "unit": UNIT,
+            "ms_per_step": round(total_ms / steps, 4), "steps": steps,
+            "tflops": round((gemm_flop + work["attention"][1]) / (total_ms / steps * 1e-3) / 1e12, 2),
+            "gemm_fp4_frac": round(gemm_flop / (gemm_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "attention_frac": round(work["attention"][1] / (stage_ms["attention"] * 1e-3) / 1e12 / att_peak, 4),
+            "ms_per_step_direct_launch": round(res["eager_ms"], 4), "stages": stages}
+
+
+# secondary workloads measured after the main line (the metric names the
+# 1024^2 T2I and I2I blocks; the multi-reference block is the stress case)
+SECONDARY = {"t2i_1024": ("i2i_1024", "multiref_1024")}
 
 
 def run_ours(args, wl):
@@ -352,122 +486,13 @@ def run_ours(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     kl.lib()
     peaks = load_peaks()
-
-    inp = block_inputs(wl)
-    T, D, H, F = wl.n_tokens, wl.hidden, wl.heads, wl.mlp_hidden
-    d = {k: v.to(dev) for k, v in inp.items()}
-    W = kl.prepare_block_weights(d["wqkv"], d["wo"], d["w1"], d["w2"])
-    cs = kl.rope_table(wl.n_text, wl.grid_h, wl.grid_w, wl.n_ref, device=dev)
-    mod = {n: d[n] for n in MOD_NAMES}
-    x = d["x"]
-    out = torch.empty_like(x)
-    ws = torch.empty(kl.block_workspace_size(T, D, H, F, wl.attn), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
-    for _ in range(args.warmup):
-        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
-    torch.cuda.synchronize()
-    st = kl.device_status()
-    if st != "KL_OK":
-        raise SystemExit(f"device status after warm-up: {st}")
-
-    def barrier():
-        rank_barrier(world, dev)
-
-    def max_over_ranks(v):
-        return rank_max(v, world, dev)
-
-    # value: the block captured once in a CUDA graph and replayed.  Every
-    # step: L2 flush, then one replay bracketed by events on the stream.  The
-    # steps are enqueued in chunks behind a short GPU sleep, so the queue is
-    # already full when the GPU reaches them and host-side enqueue time never
-    # shows up as device time.
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws)
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
-    gate_cycles = 20_000_000           # ~10 ms at B200 clocks, covers enqueueing a chunk
-    chunk = 16
-
-    def gated(n_steps, body):
-        for c0 in range(0, n_steps, chunk):
-            torch.cuda._sleep(gate_cycles)
-            for i in range(c0, min(n_steps, c0 + chunk)):
-                body(i)
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-
-    def graph_step(i):
-        flush.zero_()
-        starts[i].record()
-        graph.replay()
-        ends[i].record()
-
     clocks = ClockSampler(local)
-    barrier()
-    clocks.start()
-    gated(args.steps, graph_step)
-    barrier()
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms))
-    value = whole_job_value(world, T, args.steps, total_ms)
-
-    # per-kernel breakdown: the same steps launched directly, with the
-    # library recording an event between the stages of every step
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
-    for row in stage_ev:
-        for e in row:
-            e.record()
-
-    def eager_step(i):
-        flush.zero_()
-        kl.joint_block_forward(W, x, mod, cs, H, F, attn=wl.attn, out=out, workspace=ws, stage_events=stage_ev[i])
-
-    barrier()
-    gated(args.steps, eager_step)
-    barrier()
-    stage_ms = {s: sum(row[j].elapsed_time(row[j + 1]) for row in stage_ev) / args.steps for j, s in enumerate(STAGES)}
-    eager_ms = sum(row[0].elapsed_time(row[-1]) for row in stage_ev) / args.steps
-
-    # ---- end to end: pinned host x / mod -> device, block (graph), device ->
-    # pinned host out, all inside the timed events
-    x_h = inp["x"].pin_memory()
-    mod_h = {n: inp[n].pin_memory() for n in MOD_NAMES}
-    out_h = torch.empty_like(x_h).pin_memory()
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier()
-    def e2e_step(i):
-        flush.zero_()
-        e2e_ev[i][0].record()
-        x.copy_(x_h, non_blocking=True)
-        for n in MOD_NAMES:
-            mod[n].copy_(mod_h[n], non_blocking=True)
-        graph.replay()
-        out_h.copy_(out, non_blocking=True)
-        e2e_ev[i][1].record()
-
-    gated(args.steps, e2e_step)
-    barrier()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev))
-    del graph
-    st = kl.device_status()
-    if st != "KL_OK":
-        raise SystemExit(f"device status after timing: {st}")
-    h2d = T * D * 2 + len(MOD_NAMES) * D * 2
-    d2h = T * D * 2
-
-    work = stage_work(wl)
+    res = measure_block(kl, wl, dev, args.steps, args.warmup, flush, world, peaks, clocks=clocks, e2e=True)
+    clk = res["clk"]
     pk = tensor_peak_key(clk)
-    stages = {}
-    for s in STAGES:
-        if wl.attn != "fp8" and s == "fp8_cast":
-            continue
-        ent = roofline_entry(work[s], stage_ms[s], peaks, pk) or {}
-        ent["ms"] = round(stage_ms[s], 4)
-        stages[s] = ent
+    main = summarize(wl, res, peaks, pk, world)
+    stages = main["stages"]
     dom = max(stages, key=lambda s: stages[s]["ms"])
     roof = {k: stages[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac")}
     roof["kernel"] = dom
@@ -475,32 +500,30 @@ def run_ours(args, wl):
     kind = "burst" if pk == "bf16_tflops" else "sustained"
     roof["peak_source"] = (f"{peaks['source']} ({kind} bf16 x nominal dense ratio)" if roof["bound"] == "tensor"
                            else f"{peaks['source']} (copy)")
-    gemm_ms = sum(stage_ms[s] for s in ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm"))
-    gemm_flop = sum(work[s][1] for s in ("qkv_gemm", "out_gemm", "mlp_up_gemm", "mlp_down_gemm"))
-    fp4_peak = peaks[pk] * RATIO["fp4"]
-    att_peak = peaks[pk] * RATIO["fp8" if wl.attn == "fp8" else "bf16"]
     launches = sum(KERNELS_PER_STAGE[s] for s in stages) * args.steps
 
-    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+    line = {"metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, fp32 acc) + e4m3 attention",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, N(0,0.1) modulation)",
             "config": config_of(wl, {"parallelism": f"dp{world} (one image per GPU)" if world > 1 else "single GPU",
                                      "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
                                      "launch": "block captured once in a CUDA graph, replayed per step"}),
-            "tflops": round((gemm_flop + work["attention"][1]) / (total_ms / args.steps * 1e-3) / 1e12, 2),
-            "gemm_fp4_frac": round(gemm_flop / (gemm_ms * 1e-3) / 1e12 / fp4_peak, 4),
-            "attention_frac": round(work["attention"][1] / (stage_ms["attention"] * 1e-3) / 1e12 / att_peak, 4),
-            "roofline": roof, "stages": stages, "gpu_launches": launches,
-            "ms_per_step_direct_launch": round(eager_ms, 4),
-            "e2e": {"value": round(whole_job_value(world, T, args.steps, e2e_ms), 1), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "tflops": main["tflops"], "gemm_fp4_frac": main["gemm_fp4_frac"],
+            "attention_frac": main["attention_frac"], "roofline": roof, "stages": stages, "gpu_launches": launches,
+            "ms_per_step_direct_launch": main["ms_per_step_direct_launch"],
+            "e2e": {"value": round(whole_job_value(world, wl.n_tokens, args.steps, res["e2e_ms"]), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                    "via": "kl_joint_block_forward_host per step (pinned host x/modulation in, out back)"},
             "clocks": clk}
-    if wl.name == "t2i_1024":
-        # the metric names the 1024^2 T2I and I2I blocks: the I2I block
-        # (8,704 tokens) is measured the same way, after the main line's work
-        line["secondary"] = secondary_block(kl, WORKLOADS["i2i_1024"], dev, min(args.steps, 50), args.warmup,
-                                            flush, world)
+    sec = []
+    for name in SECONDARY.get(wl.name, ()):
+        w2 = WORKLOADS[name]
+        r2 = measure_block(kl, w2, dev, min(args.steps, 50), args.warmup, flush, world, peaks)
+        sec.append(summarize(w2, r2, peaks, pk, world))
+        torch.cuda.empty_cache()
+    if sec:
+        line["secondary"] = sec
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

@@ -99,6 +99,7 @@ _SIGS = {
     "kl_last_cuda_error": ([], ctypes.c_char_p),
     "kl_version": ([], _I),
     "kl_device_status": ([_I], _I),
+    "kl_selftest_wait_timeout": ([ctypes.c_uint64, _VP, _VP], _I),
     "kl_nvfp4_scales_bytes": ([_I64, _I64, _I], _SZ),
     "kl_quantize_workspace_size": ([], _SZ),
     "kl_quantize_nvfp4": ([_VP, _I64, _I64, _VP, _VP, _VP, _I, _VP, _SZ, _VP], _I),
@@ -120,6 +121,8 @@ _SIGS = {
                                   _I),
     "kl_block_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
     "kl_joint_block_forward": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
+    "kl_block_host_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
+    "kl_joint_block_forward_host": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
     "kl_dit_workspace_size": ([ctypes.POINTER(_DitShape)], _SZ),
     "kl_dit_step": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitWeights), ctypes.POINTER(_DitStepIO), _VP, _SZ,
                      _VP], _I),
@@ -438,6 +441,34 @@ def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, wo
     return out
 
 
+def joint_block_forward_host(weights, x_host, mod_host, rope_cs, H, F, attn="fp8", out_host=None, workspace=None,
+                             device=None):
+    """kl_joint_block_forward_host: ``x_host`` and the six ``mod_host`` vectors
+    are CPU bf16 tensors (pin them for asynchronous copies); the output comes
+    back into ``out_host`` (a CPU bf16 tensor, allocated if None) when the
+    current stream reaches the end of the call."""
+    if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+        raise ValueError("x_host: expected a contiguous CPU bf16 tensor")
+    T, D = x_host.shape
+    names = ("shift1", "scale1", "gate1", "shift2", "scale2", "gate2")
+    for n in names:
+        t = mod_host[n]
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{n}: expected a contiguous CPU bf16 tensor")
+    if out_host is None:
+        out_host = torch.empty_like(x_host, pin_memory=x_host.is_pinned())
+    device = rope_cs.device if device is None else device
+    need = lib().kl_block_host_workspace_size(T, D, H, F, ATTN[attn])
+    if workspace is None:
+        workspace = _workspace(need, device, "block_host")
+    io = _BlockIO(x_host.data_ptr(), (ctypes.c_void_p * 6)(*[mod_host[n].data_ptr() for n in names]),
+                  rope_cs.data_ptr(), T, D, H, F, ATTN[attn], out_host.data_ptr(), None, 0.0)
+    w = weights.abi()
+    _check(lib().kl_joint_block_forward_host(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
+                                             workspace.numel(), _stream()), "kl_joint_block_forward_host")
+    return out_host
+
+
 # ------------------------------------------------------------------ DiT step
 @dataclass
 class DitShape:
@@ -564,6 +595,15 @@ def dit_step_cached(shape, weights, cache, threshold, latent, text, mod_mode, mo
 def device_status(clear=True):
     """kl_device_status: synchronises and returns the status name."""
     return STATUS.get(lib().kl_device_status(1 if clear else 0), "?")
+
+
+def selftest_wait_timeout(limit_ns, waited=None):
+    """kl_selftest_wait_timeout: one warp waits on an mbarrier nothing arrives
+    on, with a bounded wait of ``limit_ns``; ``waited`` (optional CUDA int32
+    [1]) receives 0 when the wait gave up.  Asynchronous on the current stream."""
+    if waited is not None:
+        _need(waited, torch.int32, "waited")
+    _check(lib().kl_selftest_wait_timeout(int(limit_ns), _ptr(waited), _stream()), "kl_selftest_wait_timeout")
 
 
 def scales_mma_to_linear(scales, rows, cols):

@@ -40,12 +40,14 @@ static kl_status check_arch() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= kMaxDevices) return KL_ERR_ARCH;
-  if (g_arch_ok[dev] == 0) {
+  const bool cached = dev >= 0 && dev < kMaxDevices;  // devices past the cache are asked every time
+  if (!cached || g_arch_ok[dev] == 0) {
     int major = 0, minor = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    const int ok = (major == 10 && minor == 0) ? 1 : -1;
+    if (!cached) return ok == 1 ? KL_OK : KL_ERR_ARCH;
+    g_arch_ok[dev] = ok;
   }
   return g_arch_ok[dev] == 1 ? KL_OK : KL_ERR_ARCH;
 }
@@ -617,6 +619,49 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   KL_TRY(launch_gemm_nvfp4(g, s));
   mark(KL_BLOCK_STAGES);
 #undef KL_TRY
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
+// The block on host buffers: [block workspace][x][out][6 modulation vectors],
+// each piece 256-byte aligned.
+size_t kl_block_host_workspace_size(int64_t T, int64_t D, int64_t H, int64_t F, int prec) {
+  const size_t ws = kl_block_workspace_size(T, D, H, F, prec);
+  if (ws == 0) return 0;
+  return up256(ws) + 2 * up256((size_t)T * D * 2) + up256((size_t)6 * D * 2);
+}
+
+kl_status kl_joint_block_forward_host(const kl_block_weights* w, const kl_block_io* io, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  if (!w || !io || !io->x || !io->rope_cs || !io->out) return KL_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!io->mod[i]) return KL_ERR_INVALID_ARG;
+  const int64_t T = io->T, D = io->D, H = io->H, F = io->F;
+  if (io->attn_precision != KL_ATTN_FP8 && io->attn_precision != KL_ATTN_BF16) return KL_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || H > 64 || D != 128 * H || F < 128 || F % 128 || D > 8192) return KL_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = kl_block_host_workspace_size(T, D, H, F, io->attn_precision);
+  if (!workspace || ws_bytes < need) return KL_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  uint8_t* base = reinterpret_cast<uint8_t*>(workspace);
+  const size_t ws_block = up256(kl_block_workspace_size(T, D, H, F, io->attn_precision));
+  const size_t act = (size_t)T * D * 2;
+  uint8_t* x_dev = base + ws_block;
+  uint8_t* out_dev = x_dev + up256(act);
+  uint8_t* mod_dev = out_dev + up256(act);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(x_dev, io->x, act, cudaMemcpyHostToDevice, s);
+  kl_block_io dio = *io;
+  dio.x = x_dev;
+  dio.out = out_dev;
+  for (int i = 0; i < 6 && e == cudaSuccess; ++i) {
+    e = cudaMemcpyAsync(mod_dev + (size_t)i * D * 2, io->mod[i], (size_t)D * 2, cudaMemcpyHostToDevice, s);
+    dio.mod[i] = mod_dev + (size_t)i * D * 2;
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  st = kl_joint_block_forward(w, &dio, workspace, ws_block, stream);
+  if (st != KL_OK) return st;
+  e = cudaMemcpyAsync(io->out, out_dev, act, cudaMemcpyDeviceToHost, s);
   return e == cudaSuccess ? KL_OK : cuda_fail(e);
 }
 

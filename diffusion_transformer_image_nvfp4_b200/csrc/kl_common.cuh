@@ -63,9 +63,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records a timeout) if it has not after KL_WAIT_LIMIT_NS, or at once if
+// (and records a timeout) if it has not after limit_ns, or at once if
 // *abort is set by another role of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -74,12 +75,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > KL_WAIT_LIMIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(KL_DEVERR_TIMEOUT);
       *abort = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_limit(bar, parity, abort, KL_WAIT_LIMIT_NS);
 }
 
 // All 32 lanes wait together and agree on the outcome, so code after a

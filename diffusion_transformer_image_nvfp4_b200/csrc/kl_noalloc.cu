@@ -27,23 +27,68 @@ constexpr size_t kStaticScratchBytes = 256 + (size_t)kStaticScratchRows * sizeof
 // cudaGetSymbolAddress once per device (below) and passed to the kernels.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-static void* g_static_scratch_ptr[64];  // device address of g_static_scratch, per device
+// The array's device address belongs to the device's current context: a
+// cudaDeviceReset (or any teardown of the primary context) makes a new
+// context in which the array lives elsewhere.  So the address is cached per
+// device together with the id of the context it was resolved in, and
+// resolved again when that id changes.
+struct StaticScratchSlot {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+static StaticScratchSlot g_static_scratch_slot[kMaxDevices];
 static std::mutex g_static_scratch_mu;
 
-// One-time set-up on the current device: resolve the array's device address.
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+
+// id of the calling thread's current context (0 if there is none yet)
+static unsigned long long current_ctx_id() {
+  static PFN_ctx_get_current get_current = nullptr;
+  static PFN_ctx_get_id get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_ctx_get_current>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctx_get_id>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Set-up on the current device (first call, and again after the device's
+// context was replaced): resolve the array's device address with the device
+// current.  cudaGetSymbolAddress also makes the primary context current if
+// no context is yet, so the context id is read after it.
 static kl_status static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= 64) return KL_ERR_ARCH;
+  if (dev < 0 || dev >= kMaxDevices) {
+    snprintf(g_last_err, sizeof(g_last_err), "kl_ln_modulate_quantize_nvfp4_static: device index %d >= %d", dev,
+             kMaxDevices);
+    return KL_ERR_INVALID_ARG;
+  }
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_ptr[dev]) {
+  StaticScratchSlot& slot = g_static_scratch_slot[dev];
+  const unsigned long long id = current_ctx_id();
+  if (!slot.ptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
-    g_static_scratch_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_ctx_id();
   }
-  *out = g_static_scratch_ptr[dev];
+  *out = slot.ptr;
   return KL_OK;
 }
 

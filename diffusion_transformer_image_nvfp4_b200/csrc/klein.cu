@@ -7,3 +7,4 @@
 #include "kl_api.cu"
 #include "kl_noalloc.cu"
 #include "kl_dit.cu"
+#include "kl_diag.cu"

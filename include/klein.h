@@ -68,6 +68,18 @@ int kl_version(void);
  */
 kl_status kl_device_status(int clear);
 
+/*
+ * kl_selftest_wait_timeout -- exercises the failure path every kernel shares:
+ * one warp waits on an mbarrier that nothing ever arrives on, with the
+ * library's bounded wait given limit_ns (1 us .. 1 s) instead of its usual
+ * 2 s.  The wait runs out, the kernel records KL_ERR_DEVICE_TIMEOUT in the
+ * device status word (read it with kl_device_status) and returns; nothing
+ * traps and the context stays usable.  waited_out (device int, nullable)
+ * receives 0 when the wait gave up, 1 if it had completed.  Asynchronous on
+ * stream; KL_ERR_INVALID_ARG for a limit outside the range.
+ */
+kl_status kl_selftest_wait_timeout(uint64_t limit_ns, int* waited_out, void* stream);
+
 /* ------------------------------------------------------------------------
  * NVFP4 tensors
  *
@@ -173,7 +185,10 @@ kl_status kl_ln_modulate_bf16(const void* x_bf16, int64_t rows, int64_t cols, co
  *    (kl_last_cuda_error() names the limit) before anything is enqueued.
  *  - The first call on a device looks up that array's device address
  *    (cudaGetSymbolAddress) with the device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept per device with the id
+ *    of the context it belongs to and looked up again when the device's
+ *    context has been replaced (e.g. after cudaDeviceReset), so such a call
+ *    is again a first call.
  *  - All calls share the one array and it keeps the last call's contents;
  *    each call zeroes the amax word on its stream before use.  Calls that
  *    overlap on the same GPU (e.g. issued on two streams) race on it:
@@ -405,6 +420,23 @@ size_t kl_block_workspace_size(int64_t T, int64_t D, int64_t H, int64_t F, int a
  */
 kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* io,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kl_joint_block_forward_host -- kl_joint_block_forward for a caller whose
+ * activations live in host memory: io->x, io->mod[0..5] and io->out are HOST
+ * pointers (page-locked memory keeps the copies asynchronous; pageable
+ * memory makes them block the calling thread); the weights, io->rope_cs and
+ * the workspace are device memory as above.  On the stream: x and the six
+ * modulation vectors are copied into the workspace, the block runs there,
+ * and the output is copied back to io->out.  The host buffers must stay
+ * valid, and io->out unread, until the stream has reached the end of the
+ * call.  workspace: >= kl_block_host_workspace_size(...) bytes, 256-byte
+ * aligned (the block's workspace followed by x, out and the modulation
+ * vectors).
+ */
+size_t kl_block_host_workspace_size(int64_t T, int64_t D, int64_t H, int64_t F, int attn_precision);
+kl_status kl_joint_block_forward_host(const kl_block_weights* w, const kl_block_io* io,
+                                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * kl_dit_step -- one Euler step of a synthetic DiT on the block above ([P2]

@@ -53,6 +53,9 @@ def test_scale_and_workspace_sizes(L):
     assert ws >= T * 3 * D * 2 + T * 3 * D + 2 * T * D * 2 + T * F * 2 + T * F // 2
     assert L.kl_block_workspace_size(8704, 3072, 24, 9216, 1) < ws            # no FP8 copy in BF16 mode
     assert L.kl_block_workspace_size(0, 3072, 24, 9216, 0) == 0
+    host = L.kl_block_host_workspace_size(T, D, 24, F, 0)
+    assert host >= ws + 2 * T * D * 2 + 6 * D * 2                             # + x, out, modulation
+    assert L.kl_block_host_workspace_size(0, 3072, 24, 9216, 0) == 0
 
 
 def test_layout_tokens(L):
@@ -173,3 +176,9 @@ def test_sequence_parallel_pieces_validation(L):
     assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, kl.KL_AMAX_GIVEN | kl.KL_GLOBAL_SCALE_GIVEN, fake,
                                256, None) == 1
     assert L.kl_quantize_nvfp4(fake, 4, 64, fake, fake, fake, kl.KL_AMAX_GIVEN, None, 0, None) == 4
+
+
+def test_selftest_limit_is_checked_before_any_device_work(L):
+    assert L.kl_selftest_wait_timeout(0, None, None) == 1              # KL_ERR_INVALID_ARG
+    assert L.kl_selftest_wait_timeout(2_000_000_000, None, None) == 1
+    assert L.kl_selftest_wait_timeout(1_000_000, ctypes.c_void_p(2), None) == 3   # misaligned flag

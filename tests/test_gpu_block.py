@@ -83,3 +83,22 @@ def test_multiref_block_runs_and_is_deterministic():
     z = torch.zeros_like(inp["gate1"])
     c, _ = _gpu_forward(name, inp, gate1=z, gate2=z)
     np.testing.assert_array_equal(c, inp["x"].float().numpy())
+
+
+def test_host_buffer_entry_point_equals_the_device_one():
+    # kl_joint_block_forward_host: x, modulation and out in pinned host memory,
+    # copied on the stream around the same kernels -> the same bits
+    name = "tiny"
+    wl = WORKLOADS[name]
+    inp = block_inputs(name)
+    dev_out, _ = _gpu_forward(name, inp)
+    d = {k: v.cuda() for k, v in inp.items()}
+    W = kl.prepare_block_weights(d["wqkv"], d["wo"], d["w1"], d["w2"])
+    cs = kl.rope_table(wl.n_text, wl.grid_h, wl.grid_w, wl.n_ref)
+    x_h = inp["x"].pin_memory()
+    mod_h = {n: inp[n].pin_memory() for n in MOD_NAMES}
+    for _ in range(2):
+        out_h = kl.joint_block_forward_host(W, x_h, mod_h, cs, wl.heads, wl.mlp_hidden, attn=wl.attn)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(out_h.float().numpy(), dev_out)
+    assert kl.device_status() == "KL_OK"

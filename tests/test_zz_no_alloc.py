@@ -18,16 +18,28 @@ import pytest
 import torch
 
 import diffusion_transformer_image_nvfp4_b200 as kl
+from diffusion_transformer_image_nvfp4_b200 import build
 from synth import normal_bf16
 
 
-def _static_call(x, shift, scale):
-    L = kl.lib()
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return kl.lib()
+
+
+def _outputs(L, x):
     R, C = x.shape
     codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
     scales = torch.empty(L.kl_nvfp4_scales_bytes(R, C, kl.KL_SCALE_MMA), dtype=torch.uint8, device=x.device)
     gs = torch.empty(1, dtype=torch.float32, device=x.device)
     m = torch.empty_like(x)
+    return codes, scales, gs, m
+
+
+def _static_call(L, x, shift, scale, outs=None):
+    R, C = x.shape
+    codes, scales, gs, m = _outputs(L, x) if outs is None else outs
     st = L.kl_ln_modulate_quantize_nvfp4_static(
         ctypes.c_void_p(x.data_ptr()), R, C, ctypes.c_void_p(shift.data_ptr()), ctypes.c_void_p(scale.data_ptr()),
         ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(gs.data_ptr()),
@@ -37,13 +49,13 @@ def _static_call(x, shift, scale):
 
 
 @pytest.mark.gpu
-def test_static_scratch_matches_workspace_entry_point_on_two_calls():
+def test_static_scratch_matches_workspace_entry_point_on_two_calls(L):
     cases = [((4608, 3072), 1, 30.0), ((333, 512), 2, 0.05)]   # big amax first, then a small one
     for (rows, cols), seed, std in cases:
         x = normal_bf16((rows, cols), seed, std).cuda()
         shift = normal_bf16((cols,), seed + 10, 0.1).cuda()
         scale = normal_bf16((cols,), seed + 20, 0.1).cuda()
-        codes, scales, gs, m = _static_call(x, shift, scale)
+        codes, scales, gs, m = _static_call(L, x, shift, scale)
         ref, m_ref = kl.ln_modulate_quantize_nvfp4(x, shift, scale, export_m=True)
         torch.cuda.synchronize()
         assert gs.cpu().numpy().tobytes() == ref.gs.cpu().numpy().tobytes()
@@ -53,8 +65,28 @@ def test_static_scratch_matches_workspace_entry_point_on_two_calls():
     assert kl.device_status() == "KL_OK"
 
 
-def test_static_scratch_rejects_rows_beyond_its_capacity():
-    L = kl.lib()
+@pytest.mark.gpu
+def test_static_entry_point_allocates_no_device_memory(L):
+    # what the entry point is for: after a first call (which resolves the
+    # array's address and loads the kernels), further calls leave the
+    # device's free memory exactly as it was.  Inputs and outputs are made
+    # before the first reading, so torch's allocator has nothing to do.
+    x = normal_bf16((4096, 3072), 7).cuda()
+    shift = normal_bf16((3072,), 8, 0.1).cuda()
+    scale = normal_bf16((3072,), 9, 0.1).cuda()
+    outs = _outputs(L, x)
+    _static_call(L, x, shift, scale, outs)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        _static_call(L, x, shift, scale, outs)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert kl.device_status() == "KL_OK"
+
+
+def test_static_scratch_rejects_rows_beyond_its_capacity(L):
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the size check comes first
     st = L.kl_ln_modulate_quantize_nvfp4_static(fake, 32769, 512, fake, fake, fake, fake, fake, None, None)
     assert L.kl_status_string(st) == b"KL_ERR_WORKSPACE"
