@@ -94,6 +94,14 @@ def all_max(t, group=None):
     return t
 
 
+def _keep(trace, **tensors):
+    """Device copies of intermediates into ``trace`` (no-op without one)."""
+    if trace is None:
+        return
+    for k, t in tensors.items():
+        trace[k] = (t.codes.clone(), t.scales.clone(), t.gs.clone()) if isinstance(t, NVFP4) else t.clone()
+
+
 class UlyssesBlock:
     """One joint block over this rank's T/N tokens of a T-token sequence.
 
@@ -133,10 +141,13 @@ class UlyssesBlock:
         # 0 m1, 1 O, 2 m2, 3 h
         self.amax = torch.empty((4, 64), dtype=torch.float32, device=dev)
 
-    def forward(self, x, mod, rope_local, out=None):
+    def forward(self, x, mod, rope_local, out=None, trace=None):
         """x: bf16 [T/N, D] (this rank's tokens); mod: shift1 .. gate2 bf16 [D];
         rope_local: fp32 [16, T/N, 4, 2] (the rank's token columns of the
-        kl_rope_table of the whole sequence).  Returns bf16 [T/N, D]."""
+        kl_rope_table of the whole sequence).  Returns bf16 [T/N, D].
+        ``trace`` (a dict, optional): receives device copies of every
+        intermediate (m1, a1, qkv, qkv_amax, qkv8, sc8, o, oq, x1, m2, a2, h,
+        hq; NVFP4 ones as (codes, scales, gs)) for stage-by-stage checks."""
         _need(x, torch.bfloat16, "x")
         if x.shape != (self.T_loc, self.D):
             raise ValueError("x: expected this rank's [T/N, D] tokens")
@@ -150,9 +161,11 @@ class UlyssesBlock:
         ln_modulate_bf16(x, mod["shift1"], mod["scale1"], m_out=self.m, amax_out=self.amax[0])
         all_max(self.amax, g)
         quantize_nvfp4(self.m, amax_slot=self.amax[0], out=self.a)
+        _keep(trace, m1=self.m, a1=self.a)
         # 2. QKV GEMM + RoPE, per-head amax over all tokens
         gemm_nvfp4_fused(self.a, self.w.wqkv, "qkv_rope", out=self.qkv, rope_cs=rope_local, amax=self.qkv_amax)
         all_max(self.qkv_amax, g)
+        _keep(trace, qkv=self.qkv, qkv_amax=self.qkv_amax)
         # 3-4. (FP8 cast,) sequence shards -> head shards, attention on this rank's heads
         h0 = self.rank * hn
         if self.attn == "fp8":
@@ -160,6 +173,7 @@ class UlyssesBlock:
                                           self.qkv8.data_ptr(), self.sc8.data_ptr(), _stream()),
                    "kl_cast_fp8_per_head")
             heads = scatter_heads(self.qkv8, 3, H, g)
+            _keep(trace, qkv8=self.qkv8, sc8=self.sc8)
             scales = dict(sq=self.sc8[h0:h0 + hn], sk=self.sc8[H + h0:H + h0 + hn],
                           sv=self.sc8[2 * H + h0:2 * H + h0 + hn])
         else:
@@ -169,18 +183,23 @@ class UlyssesBlock:
         joint_attention(heads, heads[:, w:], heads[:, 2 * w:], self.T, hn, 3 * w, self.attn,
                         amax=self.amax[1], out=self.o_heads, **scales)
         o = gather_heads(self.o_heads, H, g)
+        _keep(trace, o=o)
         all_max(self.amax, g)
         # 5-6. NVFP4 of O, out-projection + gated residual
         quantize_nvfp4(o.contiguous(), amax_slot=self.amax[1], out=self.a)
+        _keep(trace, oq=self.a)
         gemm_nvfp4_fused(self.a, self.w.wo, "gated_residual", out=self.x1, gate=mod["gate1"], residual=x)
+        _keep(trace, x1=self.x1)
         # 7. LN2 + adaLN -> m2
         ln_modulate_bf16(self.x1, mod["shift2"], mod["scale2"], m_out=self.m, amax_out=self.amax[2])
         all_max(self.amax, g)
         quantize_nvfp4(self.m, amax_slot=self.amax[2], out=self.a)
+        _keep(trace, m2=self.m, a2=self.a)
         # 8-10. MLP-up + SwiGLU, NVFP4 of h, MLP-down + gated residual
         gemm_nvfp4_fused(self.a, self.w.w1, "swiglu", out=self.h, amax=self.amax[3])
         all_max(self.amax, g)
         quantize_nvfp4(self.h, amax_slot=self.amax[3], out=self.hq)
+        _keep(trace, h=self.h, hq=self.hq)
         gemm_nvfp4_fused(self.hq, self.w.w2, "gated_residual", out=out, gate=mod["gate2"], residual=self.x1)
         return out
 
