@@ -87,6 +87,11 @@ class _DitStepIO(ctypes.Structure):
                 ("sol_tau", ctypes.c_float)]
 
 
+class _DitViews(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_size_t), ("head_codes", ctypes.c_size_t), ("head_scales", ctypes.c_size_t),
+                ("head_gs", ctypes.c_size_t), ("velocity", ctypes.c_size_t)]
+
+
 class _DitCacheHeader(ctypes.Structure):
     _fields_ = [("num", ctypes.c_double), ("den", ctypes.c_double), ("diff", ctypes.c_float), ("hit", ctypes.c_int),
                 ("has_ref", ctypes.c_int), ("hits", ctypes.c_int), ("steps", ctypes.c_int)]
@@ -124,6 +129,7 @@ _SIGS = {
     "kl_block_host_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
     "kl_joint_block_forward_host": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
     "kl_dit_workspace_size": ([ctypes.POINTER(_DitShape)], _SZ),
+    "kl_dit_workspace_views": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitViews)], _I),
     "kl_dit_step": ([ctypes.POINTER(_DitShape), ctypes.POINTER(_DitWeights), ctypes.POINTER(_DitStepIO), _VP, _SZ,
                      _VP], _I),
     "kl_dit_cache_size": ([ctypes.POINTER(_DitShape)], _SZ),
@@ -532,6 +538,27 @@ def dit_step(shape, weights, latent, text, mod_mode, mod_joint, mod_final, rope_
     _check(lib().kl_dit_step(ctypes.byref(sh), ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
                              workspace.numel(), _stream()), "kl_dit_step")
     return latent
+
+
+def dit_views(shape, workspace):
+    """kl_dit_workspace_views as torch views into a kl_dit_step workspace
+    (uint8 CUDA tensor): tokens bf16 [T, D], head_codes uint8 [Ti, D/2],
+    head_scales uint8 (KL_SCALE_MMA layout), head_gs fp32 [1], velocity fp32
+    [Ti, 4C].  Valid after an uncached dit_step on that workspace."""
+    sh = shape.abi()
+    v = _DitViews()
+    _check(lib().kl_dit_workspace_views(ctypes.byref(sh), ctypes.byref(v)), "kl_dit_workspace_views")
+    Ti, T, D, K = shape.grid_h * shape.grid_w, shape.n_text + shape.grid_h * shape.grid_w, shape.D, 4 * shape.channels
+    nsc = lib().kl_nvfp4_scales_bytes(Ti, D, KL_SCALE_MMA)
+
+    def view(off, n, dtype):
+        return workspace[off:off + n * torch.tensor([], dtype=dtype).element_size()].view(dtype)
+
+    return {"tokens": view(v.tokens, T * D, torch.bfloat16).view(T, D),
+            "head_codes": view(v.head_codes, Ti * D // 2, torch.uint8).view(Ti, D // 2),
+            "head_scales": view(v.head_scales, nsc, torch.uint8),
+            "head_gs": view(v.head_gs, 1, torch.float32),
+            "velocity": view(v.velocity, Ti * K, torch.float32).view(Ti, K)}
 
 
 class DitCache:

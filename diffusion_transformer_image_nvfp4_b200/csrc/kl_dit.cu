@@ -383,6 +383,25 @@ size_t kl_dit_workspace_size(const kl_dit_shape* shape) {
   return dit_ws_layout(nullptr, *shape).total;
 }
 
+kl_status kl_dit_workspace_views(const kl_dit_shape* shape, kl_dit_views* out) {
+  if (!shape || !out) return KL_ERR_INVALID_ARG;
+  if (!dit_shape_ok(*shape)) return KL_ERR_UNSUPPORTED_SHAPE;
+  // the layout of a workspace placed at a nominal (aligned, non-null) base;
+  // offsets are taken from that base
+  uint8_t* const base = reinterpret_cast<uint8_t*>(uintptr_t(4096));
+  const DitWs w = dit_ws_layout(base, *shape);
+  // the blocks ping-pong between the two token buffers, starting from tok_a
+  const int n_blocks = shape->n_mode_blocks + shape->n_joint_blocks;
+  const uint16_t* fin = (n_blocks & 1) ? w.tok_b : w.tok_a;
+  auto at = [base](const void* p) { return (size_t)(reinterpret_cast<const uint8_t*>(p) - base); };
+  out->tokens = at(fin);
+  out->head_codes = at(w.fcodes);
+  out->head_scales = at(w.fscales);
+  out->head_gs = at(&w.words[4]);
+  out->velocity = at(w.v);
+  return KL_OK;
+}
+
 kl_status kl_dit_step(const kl_dit_shape* shape, const kl_dit_weights* w, const kl_dit_step_io* io, void* workspace,
                       size_t ws_bytes, void* stream) {
   kl_status r = dit_check(shape, w, io, workspace, ws_bytes);

@@ -23,6 +23,12 @@ head, so the sharded block gives the unsharded block's output bit for bit.
 The collectives are torch.distributed calls (NCCL over NVLink on GPUs; the
 data-movement helpers below also run on CPU tensors over gloo); all
 arithmetic is the library's kernels.  N must divide T and H.
+
+With a gloo process group and CUDA tensors the helpers stage through host
+memory (device -> CPU, the gloo collective, CPU -> device): the same bytes
+move and the ranks stay independent processes whose kernels never wait on
+one another, so several ranks can share one GPU (a test configuration; the
+data path is NCCL).
 """
 
 import torch
@@ -38,6 +44,21 @@ def _world(group):
 
 def _rank(group):
     return 0 if group is None else dist.get_rank(group)
+
+
+def _host_staged(t, group):
+    """True when a collective on t must go through host memory: a CUDA
+    tensor and a gloo group (gloo moves CPU tensors)."""
+    return t.is_cuda and dist.get_backend(group) == "gloo"
+
+
+def _all_to_all(recv, send, group):
+    if _host_staged(send, group):
+        r = torch.empty(recv.shape, dtype=recv.dtype)
+        dist.all_to_all_single(r, send.cpu(), group=group)
+        recv.copy_(r)
+    else:
+        dist.all_to_all_single(recv, send, group=group)
 
 
 def token_range(T, world, rank):
@@ -65,7 +86,7 @@ def scatter_heads(x, parts, heads, group=None):
     hn = heads // world
     send = x.reshape(T_loc, parts, world, hn, d).permute(2, 0, 1, 3, 4).contiguous()
     recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
+    _all_to_all(recv, send, group)
     return recv.reshape(world * T_loc, parts * hn * d)
 
 
@@ -83,14 +104,19 @@ def gather_heads(o, heads, group=None):
     T_loc = T // world
     send = o.contiguous()  # [world (destination), T/N, hn, d] in row-major order
     recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
+    _all_to_all(recv, send, group)
     return recv.reshape(world, T_loc, hn, d).permute(1, 0, 2, 3).reshape(T_loc, heads * d)
 
 
 def all_max(t, group=None):
     """In-place elementwise maximum over the ranks (identity for one rank)."""
     if _world(group) > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+        if _host_staged(t, group):
+            h = t.cpu()
+            dist.all_reduce(h, op=dist.ReduceOp.MAX, group=group)
+            t.copy_(h)
+        else:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return t
 
 

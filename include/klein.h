@@ -490,6 +490,25 @@ typedef struct kl_dit_step_io {
 } kl_dit_step_io;
 
 size_t kl_dit_workspace_size(const kl_dit_shape* shape);
+
+/*
+ * kl_dit_workspace_views -- where, inside kl_dit_step's workspace, the step
+ * leaves its intermediates, as byte offsets from the workspace start (for
+ * inspection and stage-by-stage tests; no device work).  Valid after a
+ * kl_dit_step call (not kl_dit_step_cached) until the next call that uses
+ * the workspace:
+ *   tokens       bf16 [T, D]: the sequence after the last block (the head's input)
+ *   head_codes   NVFP4 codes [grid_h*grid_w, D/2] of the head's
+ *                bf16(LN(image rows)*(1+scale_f)+shift_f)
+ *   head_scales  their scales, KL_SCALE_MMA layout
+ *   head_gs      their fp32 global scale
+ *   velocity     fp32 [grid_h*grid_w, 4*channels]: v before the Euler update
+ */
+typedef struct kl_dit_views {
+  size_t tokens, head_codes, head_scales, head_gs, velocity;
+} kl_dit_views;
+kl_status kl_dit_workspace_views(const kl_dit_shape* shape, kl_dit_views* out);
+
 kl_status kl_dit_step(const kl_dit_shape* shape, const kl_dit_weights* w, const kl_dit_step_io* io,
                       void* workspace, size_t ws_bytes, void* stream);
 

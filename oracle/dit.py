@@ -84,8 +84,7 @@ def _block(tok, i, weights, mods, shape, attn):
 
 def _head(tok, weights, mods, shape):
     """Final LN + adaLN of the image rows, NVFP4, output projection (fp64)."""
-    m = modulate(tok[shape["n_text"]:], mods["final"][0], mods["final"][1])
-    return gemm_nvfp4(nvfp4.quantize(m), nvfp4.quantize(weights["w_out"]))
+    return gemm_nvfp4(nvfp4.quantize(head_input(tok, mods, shape)), nvfp4.quantize(weights["w_out"]))
 
 
 def velocity(latent, text, weights, mods, shape, attn="exact"):
@@ -97,10 +96,22 @@ def velocity(latent, text, weights, mods, shape, attn="exact"):
     (bf16 values, kl_block_io order shift1, scale1, gate1, shift2, scale2,
     gate2); shape: dict n_text, grid_h, grid_w, channels, H.
     """
+    return _head(stack_tokens(latent, text, weights, mods, shape, attn), weights, mods, shape)
+
+
+def stack_tokens(latent, text, weights, mods, shape, attn="exact"):
+    """The token sequence [T, D] (bf16 values) after the last block of the
+    stack: the head's input (arguments as for ``velocity``)."""
     tok = _embed(latent, text, weights, shape)
     for i in range(_n_blocks(weights)):
         tok = _block(tok, i, weights, mods, shape, attn)
-    return _head(tok, weights, mods, shape)
+    return tok
+
+
+def head_input(tok, mods, shape):
+    """bf16(LN(image rows)(1 + scale_f) + shift_f): what the head encodes to
+    NVFP4 before the output projection."""
+    return modulate(np.asarray(tok)[shape["n_text"]:], mods["final"][0], mods["final"][1])
 
 
 # ---------------------------------------------------------------- Cache-DiT

@@ -123,12 +123,16 @@ class DitConfig:
 
 # c4: a 1024x1024 image -> 128x128x32 latent -> 64x64 tokens of 128 features,
 # 512 text tokens, 5 per-mode + 28 joint blocks, 16 steps; seed 3 (config
-# index - 1).  dit_tiny: the same structure at block-test sizes.
+# index - 1).  dit_tiny: the same structure at block-test sizes.  dit_wide:
+# the c4 widths (3072 hidden, 24 heads, 9216 MLP, 32 latent channels, FP8
+# attention) on a 256x256 image (16x16 tokens) and 64 text tokens, one
+# per-mode and two joint blocks, for parity at full width.
 DIT_CONFIGS = {
     c.name: c
     for c in [
         DitConfig("dit_tiny", 16, 4, 4, 32, 128, 1, 384, 1, 2, 2, "bf16", 11),
         DitConfig("dit_t2i_1024", 512, 64, 64, 32, 3072, 24, 9216, 5, 28, 16, "fp8", 3),
+        DitConfig("dit_wide", 64, 16, 16, 32, 3072, 24, 9216, 1, 2, 1, "fp8", 12),
     ]
 }
 

@@ -182,3 +182,20 @@ def test_selftest_limit_is_checked_before_any_device_work(L):
     assert L.kl_selftest_wait_timeout(0, None, None) == 1              # KL_ERR_INVALID_ARG
     assert L.kl_selftest_wait_timeout(2_000_000_000, None, None) == 1
     assert L.kl_selftest_wait_timeout(1_000_000, ctypes.c_void_p(2), None) == 3   # misaligned flag
+
+
+def test_dit_workspace_views_lie_inside_the_workspace(L):
+    sh = kl._DitShape(64, 16, 16, 32, 3072, 24, 9216, 1, 2, kl.ATTN["fp8"])
+    v = kl._DitViews()
+    assert L.kl_dit_workspace_views(ctypes.byref(sh), ctypes.byref(v)) == 0
+    size = L.kl_dit_workspace_size(ctypes.byref(sh))
+    T, Ti, D, K = 64 + 256, 256, 3072, 128
+    assert v.tokens + T * D * 2 <= size and v.velocity + Ti * K * 4 <= size
+    assert v.head_codes + Ti * D // 2 <= v.head_scales and v.head_gs % 4 == 0
+    assert all(x % 16 == 0 for x in (v.tokens, v.head_codes, v.head_scales, v.velocity))
+    # three blocks ping-pong from the first token buffer and end in the second
+    sh2 = kl._DitShape(64, 16, 16, 32, 3072, 24, 9216, 1, 1, kl.ATTN["fp8"])
+    v2 = kl._DitViews()
+    assert L.kl_dit_workspace_views(ctypes.byref(sh2), ctypes.byref(v2)) == 0
+    assert v2.tokens != v.tokens
+    assert L.kl_dit_workspace_views(None, ctypes.byref(v)) == 1

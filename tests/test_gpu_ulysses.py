@@ -90,3 +90,56 @@ def test_two_ranks_are_bit_identical_to_the_block(attn):
             p.kill()
     assert codes == [0, 0], codes
     assert sorted(q.get(timeout=10) for _ in range(2)) == [(0, True), (1, True)]
+
+
+def _staged_worker(rank, world, port, name, attn, q):
+    # every rank on cuda:0; collectives over gloo through host memory, so the
+    # ranks' kernels never wait on one another
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=120))
+    try:
+        wl = WORKLOADS[name]
+        d = block_inputs(wl)
+        W = kl.prepare_block_weights(*(d[k].to(dev) for k in ("wqkv", "wo", "w1", "w2")))
+        mod = {k: d[k].to(dev) for k in NAMES}
+        rope = kl.rope_table(wl.n_text, wl.grid_h, wl.grid_w, wl.n_ref, device=dev)
+        x = d["x"].to(dev)
+        T, H, F = wl.n_tokens, wl.heads, wl.mlp_hidden
+        ref = kl.joint_block_forward(W, x, mod, rope, H, F, attn).clone()
+        blk = ulysses.UlyssesBlock(W, T, wl.hidden, H, F, attn, group=dist.group.WORLD, device=dev)
+        got = blk.forward(x[blk.t0:blk.t1].contiguous(), mod, ulysses.local_rope(rope, blk.t0, blk.t1))
+        torch.cuda.synchronize()
+        q.put((rank, bool(torch.equal(got, ref[blk.t0:blk.t1])), kl.device_status()))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name,attn,world", [("tiny", "bf16", 2), ("tiny", "fp8", 2), ("tiny", "fp8", 4),
+                                             ("t2i_1024", "fp8", 4)])
+def test_host_staged_ranks_on_one_gpu_are_bit_identical_to_the_block(name, attn, world):
+    # the sharded path with world > 1 on one GPU: token shards, the head
+    # all-to-alls feeding the attention kernel, and the all-reduced amaxes
+    # feeding the encodes (4 ranks x 6 heads on the 4,608-token block)
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_staged_worker, args=(r, world, port, name, attn, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=600)
+    codes = [p.exitcode for p in procs]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert codes == [0] * world, codes
+    got = sorted(q.get(timeout=10) for _ in range(world))
+    assert got == [(r, True, "KL_OK") for r in range(world)], got
