@@ -202,13 +202,15 @@ def fp8_encode_heads(x):
     return e4m3_round(y), s
 
 
-def fp8_flash_rows(q8, k8, v8, c, key_tiles=None, tile=128, p_scale=16.0, tau=4.0):
+def fp8_flash_rows(q8, k8, v8, c, key_tiles=None, tile=128, p_scale=16.0, tau=4.0, return_m=False):
     """One head's flash-style pass over E4M3 operands (a reading; see below).
 
     q8 [R, d], k8 [T, d], v8 [T, d]: decoded E4M3 values (unscaled); c: the
     factor that turns q8 . k8 into log2 units of the softmax argument;
     key_tiles: the tiles of ``tile`` keys to visit, in order (default: all).
-    Returns (acc, l) with O = acc / (p_scale * l) times the V decode scale.
+    Returns (acc, l) with O = acc / (p_scale * l) times the V decode scale;
+    with ``return_m`` also the final reference maximum m, so that l * 2^m is
+    the visited keys' softmax mass sum 2^t.
 
     Steps, per visited tile: t = (q8 . k8) * c for its keys; the row's
     reference maximum m (initially -inf) is moved to the tile maximum only
@@ -244,7 +246,7 @@ def fp8_flash_rows(q8, k8, v8, c, key_tiles=None, tile=128, p_scale=16.0, tau=4.
         p = np.exp2(t - m[:, None])
         l += p.sum(axis=1)
         acc += e4m3_round(p * p_scale) @ v8[j0:j0 + tile]
-    return acc, l
+    return (acc, l, m) if return_m else (acc, l)
 
 
 def attention_fp8_emulated(q, k, v, tile=128, p_scale=16.0, tau=4.0, rows=None):
