@@ -689,6 +689,69 @@ def run_sol(args):
                       "steps": args.steps, "warmup": args.warmup, "device_status": kl.device_status()}), flush=True)
 
 
+def run_vc(args):
+    """VC-Attention repair at the 1024^2 T2I attention shape (4,608 tokens, 24
+    heads, FP8): device time of the selection + FP8 pass + BF16 pass over the
+    repaired pairs + merge, against dense FP8 attention, on seeded inputs with
+    tile structure (synth sparse_attention_qkv), inputs resident, L2 flushed
+    between steps."""
+    import diffusion_transformer_image_nvfp4_b200 as kl
+    from synth import sparse_attention_qkv
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, H = 4608, 24
+    D = H * 128
+    qkv = sparse_attention_qkv(T, H, seed=5).to(dev)
+    amax = qkv.float().abs().view(T, 3, H, 128).amax(dim=(0, 3)).reshape(-1).contiguous()
+    x8, sc = kl.cast_fp8_per_head(qkv, amax)
+    q8, k8, v8 = x8, x8[:, D:], x8[:, 2 * D:]
+    scales = dict(sq=sc[:H], sk=sc[H:2 * H], sv=sc[2 * H:])
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    l8, l16 = kl.vc_select(qkv, qkv[:, D:], T, H, 3 * D, args.vc)
+
+    def vc_step():
+        kl.vc_select(qkv, qkv[:, D:], T, H, 3 * D, args.vc)
+        kl.joint_attention_vc(q8, k8, v8, 3 * D, scales["sq"], scales["sk"], scales["sv"], qkv, qkv[:, D:],
+                              qkv[:, 2 * D:], 3 * D, T, H, l8, l16, out=out)
+
+    def dense_step():
+        kl.joint_attention(q8, k8, v8, T, H, 3 * D, "fp8", out=out, **scales)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        for _ in range(args.warmup):
+            graph.replay()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            ms.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in ms])
+
+    t_vc, t_dense = timed(vc_step), timed(dense_step)
+    repaired = int((l16[:, 0::2, 0] if l16.shape[1] > 1 else l16[:, :, 0]).sum().item())
+    print(json.dumps({"metric": "VC-Attention device time (selection + FP8 pass + repaired BF16 pass + merge), "
+                                "1024^2 T2I shape", "value": round(t_vc * 1000, 1), "unit": "us",
+                      "higher_is_better": False, "dense_fp8_us": round(t_dense * 1000, 1),
+                      "overhead": round(t_vc / t_dense, 3), "budget": args.vc, "repaired_pairs": repaired,
+                      "pairs": int(H * l8.shape[1] * (l8.shape[2] - 1)),
+                      "config": {"workload": "vc_attention_t2i_1024", "tokens": T, "heads": H, "query_block": 256,
+                                 "key_tile": 128, "inputs": "synth.sparse_attention_qkv(seed 5)",
+                                 "launch": "each leg captured in a CUDA graph, replayed per step",
+                                 "l2": "flushed between timed steps (256 MiB write, outside the timed events)"},
+                      "steps": args.steps, "warmup": args.warmup, "device_status": kl.device_status()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -703,6 +766,8 @@ def main():
                     help="--dit: Cache-DiT residual-difference threshold (e.g. 0.24); default off")
     ap.add_argument("--sol", type=float, default=None,
                     help="time Sol-Attention (selection + sparse attention) at this tau against dense attention")
+    ap.add_argument("--vc", type=float, default=None,
+                    help="time VC-Attention repair (selection + both passes + merge) at this budget against dense")
     ap.add_argument("--sol-tau", type=float, default=0.0, help="--dit: Sol-Attention tau for every block (0: dense)")
     ap.add_argument("--sol-dense-steps", type=int, default=0, help="--dit: the first N steps stay dense")
     ap.add_argument("--mods", choices=("independent", "smooth"), default="independent",
@@ -716,6 +781,9 @@ def main():
         return
     if args.sol is not None:
         run_sol(args)
+        return
+    if args.vc is not None:
+        run_vc(args)
         return
     if args.impl == "reference":
         run_reference(args, wl)

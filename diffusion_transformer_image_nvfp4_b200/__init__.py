@@ -65,7 +65,8 @@ class _BlockIO(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("mod", ctypes.c_void_p * 6), ("rope_cs", ctypes.c_void_p),
                 ("T", ctypes.c_int64), ("D", ctypes.c_int64), ("H", ctypes.c_int64), ("F", ctypes.c_int64),
                 ("attn_precision", ctypes.c_int), ("out", ctypes.c_void_p),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("sol_tau", ctypes.c_float)]
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("sol_tau", ctypes.c_float),
+                ("vc_budget", ctypes.c_float)]
 
 
 class _DitShape(ctypes.Structure):
@@ -124,6 +125,11 @@ _SIGS = {
     "kl_sol_select": ([_VP, _VP, _I64, _VP, _VP, _I64, _I64, _I, ctypes.c_float, _VP, _VP, _SZ, _VP], _I),
     "kl_joint_attention_sparse": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _I64, _I64, _I64, _I, _VP, _VP, _VP, _VP],
                                   _I),
+    "kl_vc_workspace_size": ([_I64, _I64], _SZ),
+    "kl_vc_select": ([_VP, _VP, _I64, _I64, _I64, ctypes.c_float, _VP, _VP, _VP, _SZ, _VP], _I),
+    "kl_vc_attention_workspace_size": ([_I64, _I64], _SZ),
+    "kl_joint_attention_vc": ([_VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _VP, _VP,
+                               _VP, _VP, _VP, _SZ, _VP], _I),
     "kl_block_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
     "kl_joint_block_forward": ([ctypes.POINTER(_BlockWeights), ctypes.POINTER(_BlockIO), _VP, _SZ, _VP], _I),
     "kl_block_host_workspace_size": ([_I64, _I64, _I64, _I64, _I], _SZ),
@@ -390,6 +396,32 @@ def joint_attention_sparse(q, k, v, T, H, ld, kv_list, precision="fp8", sq=None,
     return out
 
 
+def vc_select(q, k, T, H, ld, budget):
+    """kl_vc_select on bf16 q, k: (list_fp8 int32 [H, ceil(T/256), n_kt + 1]
+    of the tiles that are not repaired, list_bf16 int32 [H, ceil(T/128), n_kt +
+    1] of the repaired ones), each row the count then ascending tile indices."""
+    nkt = -(-T // 128)
+    l8 = torch.zeros((H, -(-T // 256), nkt + 1), dtype=torch.int32, device=q.device)
+    l16 = torch.zeros((H, -(-T // 128), nkt + 1), dtype=torch.int32, device=q.device)
+    ws = _workspace(lib().kl_vc_workspace_size(T, H), q.device, "vc")
+    _check(lib().kl_vc_select(q.data_ptr(), k.data_ptr(), ld, T, H, float(budget), l8.data_ptr(), l16.data_ptr(),
+                              ws.data_ptr(), ws.numel(), _stream()), "kl_vc_select")
+    return l8, l16
+
+
+def joint_attention_vc(q8, k8, v8, ld8, sq, sk, sv, q, k, v, ld, T, H, list_fp8, list_bf16, amax=None, out=None):
+    """kl_joint_attention_vc: FP8 attention (E4M3 q8, k8, v8 with per-head
+    scales) with the pairs of list_bf16 computed from the bf16 q, k, v."""
+    if out is None:
+        out = torch.empty((T, H * 128), dtype=torch.bfloat16, device=q8.device)
+    ws = _workspace(lib().kl_vc_attention_workspace_size(T, H), q8.device, "vc_att")
+    _check(lib().kl_joint_attention_vc(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), ld8, sq.data_ptr(), sk.data_ptr(),
+                                       sv.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), ld, T, H, 128,
+                                       list_fp8.data_ptr(), list_bf16.data_ptr(), out.data_ptr(), _ptr(amax),
+                                       ws.data_ptr(), ws.numel(), _stream()), "kl_joint_attention_vc")
+    return out
+
+
 # ---------------------------------------------------------------- block
 @dataclass
 class BlockWeights:
@@ -417,12 +449,13 @@ BLOCK_STAGES = ("ln1", "qkv_gemm", "fp8_cast", "attention", "quant_o", "out_gemm
 
 
 def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, workspace=None, stage_events=None,
-                        sol_tau=0.0):
+                        sol_tau=0.0, vc_budget=0.0):
     """kl_joint_block_forward.  ``mod`` maps shift1, scale1, gate1, shift2,
     scale2, gate2 to bf16 [D] CUDA tensors.  ``stage_events`` (optional): a list
     of len(BLOCK_STAGES)+1 recorded torch.cuda.Event(enable_timing=True); the
     library re-records them around each stage on the current stream.
-    ``sol_tau`` > 0: Sol-Attention tile skipping at that threshold."""
+    ``sol_tau`` > 0: Sol-Attention tile skipping at that threshold.
+    ``vc_budget`` > 0: VC-Attention repair of that fraction of the FP8 tile pairs."""
     _need(x, torch.bfloat16, "x")
     T, D = x.shape
     names = ("shift1", "scale1", "gate1", "shift2", "scale2", "gate2")
@@ -440,7 +473,7 @@ def joint_block_forward(weights, x, mod, rope_cs, H, F, attn="fp8", out=None, wo
         ev = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
     io = _BlockIO(x.data_ptr(), (ctypes.c_void_p * 6)(*[mod[n].data_ptr() for n in names]), rope_cs.data_ptr(),
                   T, D, H, F, ATTN[attn], out.data_ptr(), ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p)),
-                  float(sol_tau))
+                  float(sol_tau), float(vc_budget))
     w = weights.abi()
     _check(lib().kl_joint_block_forward(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(), workspace.numel(),
                                         _stream()), "kl_joint_block_forward")
@@ -468,7 +501,7 @@ def joint_block_forward_host(weights, x_host, mod_host, rope_cs, H, F, attn="fp8
     if workspace is None:
         workspace = _workspace(need, device, "block_host")
     io = _BlockIO(x_host.data_ptr(), (ctypes.c_void_p * 6)(*[mod_host[n].data_ptr() for n in names]),
-                  rope_cs.data_ptr(), T, D, H, F, ATTN[attn], out_host.data_ptr(), None, 0.0)
+                  rope_cs.data_ptr(), T, D, H, F, ATTN[attn], out_host.data_ptr(), None, 0.0, 0.0)
     w = weights.abi()
     _check(lib().kl_joint_block_forward_host(ctypes.byref(w), ctypes.byref(io), workspace.data_ptr(),
                                              workspace.numel(), _stream()), "kl_joint_block_forward_host")

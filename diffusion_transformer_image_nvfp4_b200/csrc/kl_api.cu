@@ -409,6 +409,104 @@ kl_status kl_joint_attention_sparse(const void* q, const void* k, const void* v,
   return e == cudaSuccess ? KL_OK : cuda_fail(e);
 }
 
+// ------------------------------------------------------------ VC-Attention
+size_t kl_vc_workspace_size(int64_t T, int64_t H) {
+  if (T < 1 || H < 1) return 0;
+  return vc_select_workspace_bytes(T, H);
+}
+
+kl_status kl_vc_select(const void* q, const void* k, int64_t ld, int64_t T, int64_t H, float budget, int* list_fp8,
+                       int* list_bf16, void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k || !list_fp8 || !list_bf16) return KL_ERR_INVALID_ARG;
+  if (!(budget >= 0.f && budget <= 1.f)) return KL_ERR_INVALID_ARG;  // also rejects NaN
+  if (T < 1 || H < 1 || H > 65535 || ld < H * 128 || ld % 64 || (T + 127) / 128 > 12 * 1024)
+    return KL_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || ws_bytes < kl_vc_workspace_size(T, H)) return KL_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(list_fp8, 4) || !aligned(list_bf16, 4) ||
+      !aligned(workspace, 256))
+    return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  cudaError_t e = launch_vc_select(q, k, ld, T, H, budget, list_fp8, list_bf16, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
+// [ml8: float2 T*H][ml16: float2 T*H][o16: fp32 T*H*128]
+size_t kl_vc_attention_workspace_size(int64_t T, int64_t H) {
+  if (T < 1 || H < 1) return 0;
+  return 2 * up256((size_t)T * H * sizeof(float2)) + up256((size_t)T * H * 128 * sizeof(float));
+}
+
+static cudaError_t vc_attention(const AttnArgs& a8, const void* q, const void* k, const void* v, int64_t ld,
+                                const int* list16, uint8_t* ws, cudaStream_t s) {
+  const int64_t T = a8.T, H = a8.H;
+  float2* ml8 = reinterpret_cast<float2*>(ws);
+  float2* ml16 = reinterpret_cast<float2*>(ws + up256((size_t)T * H * sizeof(float2)));
+  float* o16 = reinterpret_cast<float*>(ws + 2 * up256((size_t)T * H * sizeof(float2)));
+  AttnArgs f = a8;  // the FP8 pass over the tiles that are not repaired
+  f.amax = nullptr;
+  f.ml_out = ml8;
+  f.empty_ok = 1;
+  cudaError_t e = launch_attention(f, s);
+  if (e != cudaSuccess) return e;
+  AttnArgs b{};  // the BF16 pass over the repaired tiles
+  b.q = q;
+  b.k = k;
+  b.v = v;
+  b.ld = ld;
+  b.T = T;
+  b.H = H;
+  b.fp8 = 0;
+  b.out = a8.out;
+  b.kv_list = list16;
+  b.ml_out = ml16;
+  b.o32 = o16;
+  b.empty_ok = 1;
+  if ((e = launch_attention(b, s)) != cudaSuccess) return e;
+  if ((e = launch_vc_merge(a8.out, o16, ml8, ml16, T, H, s)) != cudaSuccess) return e;
+  if (!a8.amax) return cudaSuccess;
+  // max |O| of the merged output, max-accumulated into amax
+  return launch_pdl(amax_bf16_kernel, dim3(grid_for(T * H * 16, 256)), dim3(256), 0, s,
+                    reinterpret_cast<const uint4*>(a8.out), T * H * 16, a8.amax);
+}
+
+kl_status kl_joint_attention_vc(const void* q8, const void* k8, const void* v8, int64_t ld8, const float* sq,
+                                const float* sk, const float* sv, const void* q, const void* k, const void* v,
+                                int64_t ld, int64_t T, int64_t H, int64_t head_dim, const int* list_fp8,
+                                const int* list_bf16, void* out, float* amax_out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !q || !k || !v || !list_fp8 || !list_bf16 || !out)
+    return KL_ERR_INVALID_ARG;
+  if (head_dim != 128 || T < 1 || H < 1 || H > 65535 || T > (int64_t)1 << 31 || ld8 < H * 128 || ld8 % 64 ||
+      ld < H * 128 || ld % 64)
+    return KL_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || ws_bytes < kl_vc_attention_workspace_size(T, H)) return KL_ERR_WORKSPACE;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(q, 16) || !aligned(k, 16) ||
+      !aligned(v, 16) || !aligned(out, 16) || !aligned(list_fp8, 4) || !aligned(list_bf16, 4) ||
+      !aligned(workspace, 256) || (amax_out && !aligned(amax_out, 4)))
+    return KL_ERR_MISALIGNED;
+  kl_status st = check_arch();
+  if (st != KL_OK) return st;
+  AttnArgs a{};
+  a.q = q8;
+  a.k = k8;
+  a.v = v8;
+  a.ld = ld8;
+  a.sq = sq;
+  a.sk = sk;
+  a.sv = sv;
+  a.T = T;
+  a.H = H;
+  a.fp8 = 1;
+  a.out = out;
+  a.amax = amax_out;
+  a.kv_list = list_fp8;
+  cudaError_t e = vc_attention(a, q, k, v, ld, list_bf16, reinterpret_cast<uint8_t*>(workspace),
+                               reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KL_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------ block driver
 // Workspace layout (each piece 256-byte aligned):
 //   words  : amax[0..3] (O at 1, h at 3), gs[4..7], qkv amax [3H], fp8 scales [3H],
@@ -428,6 +526,9 @@ struct BlockWs {
   uint16_t *qkv, *o, *x1, *h;
   void* sol_ws;   // Sol-Attention block means
   int* sol_list;  // Sol-Attention key-tile lists
+  void* vc_ws;    // VC-Attention: shares and marks, the two tile lists, the partial results
+  int *vc_list8, *vc_list16;
+  uint8_t* vc_att;
   size_t total;
 };
 static BlockWs block_ws_layout(uint8_t* base, int64_t T, int64_t D, int64_t H, int64_t F, int prec) {
@@ -452,6 +553,12 @@ static BlockWs block_ws_layout(uint8_t* base, int64_t T, int64_t D, int64_t H, i
   w.hscales = take((size_t)Tp * F / 16);
   w.sol_ws = take(sol_workspace_bytes(T, H, prec == KL_ATTN_FP8));
   w.sol_list = reinterpret_cast<int*>(take(sol_list_ints(T, H, prec == KL_ATTN_FP8) * sizeof(int)));
+  if (prec == KL_ATTN_FP8) {
+    w.vc_ws = take(vc_select_workspace_bytes(T, H));
+    w.vc_list8 = reinterpret_cast<int*>(take(sol_list_ints(T, H, true) * sizeof(int)));
+    w.vc_list16 = reinterpret_cast<int*>(take(sol_list_ints(T, H, false) * sizeof(int)));
+    w.vc_att = take(kl_vc_attention_workspace_size(T, H));
+  }
   w.total = off;
   return w;
 }
@@ -470,6 +577,8 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
   if (io->attn_precision != KL_ATTN_FP8 && io->attn_precision != KL_ATTN_BF16) return KL_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || H > 64 || D != 128 * H || F < 128 || F % 128 || D > 8192) return KL_ERR_UNSUPPORTED_SHAPE;
   if (io->out == io->x) return KL_ERR_INVALID_ARG;
+  if (!(io->vc_budget >= 0.f && io->vc_budget <= 1.f)) return KL_ERR_INVALID_ARG;  // also rejects NaN
+  if (io->vc_budget > 0.f && (io->attn_precision != KL_ATTN_FP8 || io->sol_tau > 0.f)) return KL_ERR_INVALID_ARG;
   kl_status st = KL_OK;
   const kl_nvfp4_tensor* ops[4] = {&w->wqkv, &w->wo, &w->w1, &w->w2};
   for (auto* t : ops)
@@ -551,7 +660,13 @@ kl_status kl_joint_block_forward(const kl_block_weights* w, const kl_block_io* i
     KL_TRY(launch_sol_select(a.q, a.k, a.ld, a.sq, a.sk, T, H, a.fp8 != 0, io->sol_tau, ws.sol_list, ws.sol_ws, s));
     a.kv_list = ws.sol_list;
   }
-  KL_TRY(launch_attention(a, s));
+  if (io->vc_budget > 0.f) {  // VC-Attention: repaired tile pairs from the bf16 q, k, v
+    KL_TRY(launch_vc_select(ws.qkv, ws.qkv + D, 3 * D, T, H, io->vc_budget, ws.vc_list8, ws.vc_list16, ws.vc_ws, s));
+    a.kv_list = ws.vc_list8;
+    KL_TRY(vc_attention(a, ws.qkv, ws.qkv + D, ws.qkv + 2 * D, 3 * D, ws.vc_list16, ws.vc_att, s));
+  } else {
+    KL_TRY(launch_attention(a, s));
+  }
   mark(4);
   // 5. O -> NVFP4 (gs from the attention amax)
   KL_TRY(launch_quantize(ws.o, T, D, ws.acodes, ws.ascales, &gs[1], &amax[1], 1, s));

@@ -51,6 +51,10 @@ struct AttnParams {
   uint16_t* out;
   float* amax;
   const int* kv_list;  // nullable: per (head, query block) [count, tile indices...], n_kv + 1 ints
+  // partial results (VC-Attention repair): all nullable / 0 by default
+  float2* ml_out;      // [T, H]: per row the reference maximum m and the mass l (sum 2^(t-m) of the visited keys)
+  float* o32;          // [T, H*128] fp32: O written here (normalised, FP8: times s_v) instead of bf16 to out
+  int empty_ok;        // a list count of 0 is allowed: the CTA only writes ml_out = (-inf, 0) for its rows
 };
 
 template <bool FP8>
@@ -150,7 +154,9 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   int n = p.n_kv;
   if constexpr (SPARSE) {
     n = __ldg(kv_tiles);
-    n = n < 1 ? 1 : (n > p.n_kv ? p.n_kv : n);  // at least one tile: the last P.V signals the epilogue
+    // at least one tile (the last P.V signals the epilogue), unless empty lists are allowed
+    const int lo = p.empty_ok ? 0 : 1;
+    n = n < lo ? lo : (n > p.n_kv ? p.n_kv : n);
   }
   uint8_t* q_smem = smem + C::Q_OFF;
   uint8_t* kv_smem = smem + C::KV_OFF;
@@ -423,15 +429,30 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
     float lsum = 0.f;
 #pragma unroll
     for (int q = 0; q < C::SPLIT; ++q) lsum += lsm[(t * C::SPLIT + q) * 128 + r];
-    // epilogue: O / l (FP8: times s_v), bf16, tensor amax
+    // epilogue: O / l (FP8: times s_v), bf16 (or fp32), tensor amax
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) ok = warp_wait(&o_last[t], 0, abort_flag);
+    if (ok && n > 0) ok = warp_wait(&o_last[t], 0, abort_flag);
     const int64_t row = ((int64_t)qblk * QT + t) * 128 + r;
-    const bool valid_row = ok && row < p.T;
+    const bool valid_row = ok && n > 0 && row < p.T;
+    if (p.ml_out && part == 0 && ok && row < p.T)  // the mass of the visited keys: lsum / P_SCALE * 2^m
+      p.ml_out[row * p.H + h] = n > 0 ? make_float2(m, lsum * (1.0f / C::P_SCALE)) : make_float2(-INFINITY, 0.f);
     float scale = 1.0f / lsum;  // l sums p * P_SCALE, so this also undoes P_SCALE
     if (FP8) scale *= __ldg(p.sv + h);
     float amax = 0.f;
-    if (ok) {
+    if (ok && n > 0 && p.o32) {
+      tc_fence_after();
+      float4* dst = reinterpret_cast<float4*>(p.o32 + row * (int64_t)p.H * 128 + h * 128 + part * COLS);
+#pragma unroll 1
+      for (int cc = 0; cc < COLS / 32; ++cc) {
+        float o[32];
+        tmem_ld32(o_tmem + cc * 32, o);
+        if (valid_row)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[cc * 8 + q] = make_float4(o[4 * q] * scale, o[4 * q + 1] * scale, o[4 * q + 2] * scale,
+                                          o[4 * q + 3] * scale);
+      }
+    } else if (ok && n > 0) {
       tc_fence_after();
       uint4* dst = reinterpret_cast<uint4*>(p.out + row * (int64_t)p.H * 128 + h * 128 + part * COLS);
 #pragma unroll 1
@@ -488,6 +509,9 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
   p.out = reinterpret_cast<uint16_t*>(a.out);
   p.amax = a.amax;
   p.kv_list = a.kv_list;
+  p.ml_out = a.ml_out;
+  p.o32 = a.o32;
+  p.empty_ok = a.empty_ok;
   const int qblocks = (int)((a.T + 128 * C::QT - 1) / (128 * C::QT));
   dim3 grid((unsigned)qblocks, (unsigned)a.H);
   auto kern = a.kv_list ? attn_kernel<FP8, true> : attn_kernel<FP8, false>;

@@ -81,6 +81,9 @@ struct AttnArgs {
   void* out;   // bf16 [T, H*128]
   float* amax; // nullable
   const int* kv_list = nullptr;  // nullable: Sol-Attention key-tile lists (kl_sol_select layout)
+  float2* ml_out = nullptr;      // nullable: per (row, head) reference maximum m and mass l (partial results)
+  float* o32 = nullptr;          // nullable: fp32 output instead of out (partial results)
+  int empty_ok = 0;              // kv_list counts of 0 allowed (the CTA writes only ml_out)
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
@@ -90,6 +93,14 @@ size_t sol_list_ints(int64_t T, int64_t H, bool fp8);
 size_t sol_workspace_bytes(int64_t T, int64_t H, bool fp8);
 cudaError_t launch_sol_select(const void* q, const void* k, int64_t ld, const float* sq, const float* sk, int64_t T,
                               int64_t H, bool fp8, float tau, int* list, void* ws, cudaStream_t s);
+
+// VC-Attention repair (kl_vc.cu)
+size_t vc_select_workspace_bytes(int64_t T, int64_t H);
+int64_t vc_repair_count(int64_t T, float budget);  // repaired pairs per head
+cudaError_t launch_vc_select(const void* q, const void* k, int64_t ld, int64_t T, int64_t H, float budget,
+                             int* list8, int* list16, void* ws, cudaStream_t s);
+cudaError_t launch_vc_merge(void* out, const float* o16, const float2* ml8, const float2* ml16, int64_t T,
+                            int64_t H, cudaStream_t s);
 
 // tensor maps (kl_api.cu)
 // 2D tensor map, box_inner x box_outer elements; swizzle_bytes 128, 64 or 0 (none)

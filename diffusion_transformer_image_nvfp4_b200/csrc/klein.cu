@@ -4,6 +4,7 @@
 #include "kl_gemm.cu"
 #include "kl_attn.cu"
 #include "kl_sparse.cu"
+#include "kl_vc.cu"
 #include "kl_api.cu"
 #include "kl_noalloc.cu"
 #include "kl_dit.cu"

@@ -362,6 +362,53 @@ kl_status kl_joint_attention_sparse(const void* q, const void* k, const void* v,
                                     int64_t head_dim, int precision, const int* kv_list, void* out,
                                     float* amax_out, void* stream);
 
+/*
+ * VC-Attention repair ([P1] "Optimizing FLUX 3 Image Klein inference on
+ * NVIDIA Blackwell GPUs", How it works: VC-Attention adds a repair budget that
+ * corrects the quantization errors of FP8 attention; Key details: a repair
+ * budget of 0.005).  Readings (the pages give no more): the unit of repair is
+ * the FP8 attention's tile pair, a query block of 256 rows against a key tile
+ * of 128 keys, per head; budget b repairs R = floor(b * n_qb * n_kt) of a
+ * head's n_qb * n_kt pairs (n_qb = ceil(T/256), n_kt = ceil(T/128)): those
+ * with the largest estimated share of their query block's attention,
+ *   w(b, j) = 2^(s_hat(b,j) - max_j') / sum_j' 2^(s_hat(b,j') - max_j'),
+ *   s_hat = (qbar . kbar) * log2(e)/sqrt(128),
+ * qbar / kbar the means of the block's bf16 query rows / the tile's bf16 key
+ * rows (valid rows only); equal shares go to the lower (b, j) in row-major
+ * order.  Shares are fp32, so pairs whose shares lie within fp32 rounding of
+ * the R-th largest may go either way.  A repaired pair is computed from the
+ * bf16 q, k, v: the query block's output is the exact merge of the FP8
+ * attention over its other tiles and the BF16 attention over its repaired
+ * tiles, O = (O_8 W_8 + O_16 W_16) / (W_8 + W_16), W the softmax mass of
+ * each part.
+ *
+ * kl_vc_select: q, k bf16 [T, H, 128] (row stride ld, a multiple of 64;
+ * 16-byte aligned), budget in [0, 1].  list_fp8 (kl_sol_list_ints(T, H,
+ * KL_ATTN_FP8) ints): per (head, 256-row block) the tiles that are not
+ * repaired; list_bf16 (kl_sol_list_ints(T, H, KL_ATTN_BF16) ints): per (head,
+ * 128-row block) the repaired tiles of its 256-row block; both ascending, in
+ * the kl_sol_select layout, counts may be 0.  workspace >=
+ * kl_vc_workspace_size(T, H) bytes, 256-byte aligned.
+ *
+ * kl_joint_attention_vc: q8, k8, v8 E4M3 (row stride ld8) with scales sq, sk,
+ * sv as for kl_joint_attention_fp8, and q, k, v their bf16 values (row stride
+ * ld); the two lists from kl_vc_select.  out bf16 [T, H*128]; amax_out
+ * (nullable) max-accumulates max|out| (caller zero-fills).  workspace >=
+ * kl_vc_attention_workspace_size(T, H) bytes, 256-byte aligned (per row and
+ * head the reference maximum and mass of both parts, and the BF16 part's
+ * fp32 output).  With budget 0 the result is kl_joint_attention_fp8's bit for
+ * bit.
+ */
+size_t kl_vc_workspace_size(int64_t T, int64_t H);
+kl_status kl_vc_select(const void* q, const void* k, int64_t ld, int64_t T, int64_t H, float budget, int* list_fp8,
+                       int* list_bf16, void* workspace, size_t ws_bytes, void* stream);
+size_t kl_vc_attention_workspace_size(int64_t T, int64_t H);
+kl_status kl_joint_attention_vc(const void* q8, const void* k8, const void* v8, int64_t ld8, const float* scale_q,
+                                const float* scale_k, const float* scale_v, const void* q, const void* k,
+                                const void* v, int64_t ld, int64_t T, int64_t H, int64_t head_dim,
+                                const int* list_fp8, const int* list_bf16, void* out, float* amax_out,
+                                void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * The joint block
  * ---------------------------------------------------------------------- */
@@ -387,6 +434,9 @@ typedef struct kl_block_io {
                            attention; > 0 = each query block visits only the key
                            tiles kl_sol_select keeps at this tau (selection runs
                            inside the attention stage)                          */
+  float vc_budget;      /* VC-Attention repair budget in [0, 1]: 0 (default) = off;
+                           > 0 = FP8 attention only (not with sol_tau), the pairs
+                           kl_vc_select picks are computed from the bf16 q, k, v */
 } kl_block_io;
 
 /* Stages of kl_joint_block_forward, in launch order (stage_events index). */

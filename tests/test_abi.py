@@ -199,3 +199,14 @@ def test_dit_workspace_views_lie_inside_the_workspace(L):
     assert L.kl_dit_workspace_views(ctypes.byref(sh2), ctypes.byref(v2)) == 0
     assert v2.tokens != v.tokens
     assert L.kl_dit_workspace_views(None, ctypes.byref(v)) == 1
+
+
+def test_vc_argument_checks(L):
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.kl_vc_workspace_size(4608, 24) > 0 and L.kl_vc_workspace_size(0, 24) == 0
+    assert L.kl_vc_attention_workspace_size(4608, 24) >= 2 * 4608 * 24 * 8 + 4608 * 24 * 128 * 4
+    ws = L.kl_vc_workspace_size(1000, 2)
+    sel = lambda budget: L.kl_vc_select(fake, fake, 768, 1000, 2, budget, fake, fake, fake, ws, None)
+    assert sel(float("nan")) == 1 and sel(-0.1) == 1 and sel(1.5) == 1          # KL_ERR_INVALID_ARG
+    assert L.kl_vc_select(fake, fake, 100, 1000, 2, 0.1, fake, fake, fake, ws, None) == 2   # ld too small
+    assert L.kl_vc_select(fake, fake, 768, 1000, 2, 0.1, fake, fake, fake, ws - 1, None) == 4  # workspace
