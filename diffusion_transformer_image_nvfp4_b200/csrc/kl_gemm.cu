@@ -46,6 +46,7 @@ struct GemmParams {
   const uint16_t* residual;
   float* amax;
   int num_m, num_tiles, num_kt, kbn;  // kbn = K / 64
+  int res_prefetch;                   // 2-SM kernel: L2 prefetch of each tile's residual rows
 };
 
 // BN: output tile width (256 or 128).  KS: 64-wide K steps per smem stage
@@ -165,6 +166,61 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
     }
     amax = warp_max(valid ? amax : 0.f);
     if (lane == 0) atomic_max_nonneg(p.amax, amax);
+  } else if (BN == 256 && p.epi == KL_EPI_QKV_ROPE) {
+    // two heads per tile (columns n0.. and n0 + 128..), each in its own
+    // region (q, k or v); this thread holds the columns of pairs
+    // [32*half, 32*half + 32) of both: v[0..63] head A, v[64..127] head B
+    int region[2], head[2];
+    float hmax[2] = {0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int64_t ne = n0 + e * 128;
+      region[e] = (int)(ne / D);
+      head[e] = (int)((ne - (int64_t)region[e] * D) >> 7);
+    }
+    const bool rope = region[0] < 2 || region[1] < 2;
+    // table: groups of 4 pairs per token ([16][M][4] of (c, s)); pair
+    // 32*half + c/2 + 4*g4 + u of chunk c is group 8*half + c/8 + g4
+    const float* cs =
+        reinterpret_cast<const float*>(p.rope_cs) + ((int64_t)(8 * half) * p.M + (valid ? row : 0)) * 8;
+#pragma unroll
+    for (int c = 0; c < 64; c += 32) {
+      if (rope) {
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float t[8];
+          // (not volatile: a read-only load the compiler may schedule early)
+          asm("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+              : "=f"(t[0]), "=f"(t[1]), "=f"(t[2]), "=f"(t[3]), "=f"(t[4]), "=f"(t[5]), "=f"(t[6]), "=f"(t[7])
+              : "l"(cs + ((int64_t)(c >> 3) + g4) * p.M * 8));
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            if (region[e] < 2) {
+              float* w = v + e * 64 + c + 8 * g4;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float a0 = w[2 * u], b0 = w[2 * u + 1];
+                w[2 * u] = a0 * t[2 * u] - b0 * t[2 * u + 1];
+                w[2 * u + 1] = a0 * t[2 * u + 1] + b0 * t[2 * u];
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float* w = v + e * 64 + c;
+        hmax[e] = fmaxf(hmax[e], round_bf16x32(*reinterpret_cast<float(*)[32]>(w)));
+        if (valid)
+          store_bf16x32(reinterpret_cast<uint16_t*>(p.out) + row * p.N + n0 + e * 128 + 64 * half + c,
+                        *reinterpret_cast<float(*)[32]>(w));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float m = warp_max(valid ? hmax[e] : 0.f);
+      if (lane == 0) atomic_max_nonneg(p.amax + region[e] * H + head[e], m);
+    }
   } else {
     // QKV: a thread's HALF (<= 128) columns lie in one head of one region
     // (heads are 128 columns, n0 + half*HALF is a multiple of HALF)
@@ -239,9 +295,17 @@ template <int BN>
 __device__ __forceinline__ void epilogue_drain(const GemmParams& p, uint32_t tbase, int half, float (&v)[BN / 2]) {
   constexpr int HALF = BN / 2;
   if constexpr (BN == 256) {
-    // columns [128*half, 128*half + 128): for SwiGLU that is exactly one
-    // 64-gate + 64-up row group, already in the order used by the epilogue
-    tmem_ld128(tbase + half * 128, v);
+    if (p.epi == KL_EPI_QKV_ROPE) {
+      // the tile holds two heads: this thread takes rotation pairs
+      // [32*half, 32*half + 32) of both (columns 64*half.. and 128 + 64*half..),
+      // so the RoPE table entries it loads serve both heads
+      tmem_ld64(tbase + half * 64, *reinterpret_cast<float(*)[64]>(v));
+      tmem_ld64(tbase + 128 + half * 64, *reinterpret_cast<float(*)[64]>(v + 64));
+    } else {
+      // columns [128*half, 128*half + 128): for SwiGLU that is exactly one
+      // 64-gate + 64-up row group, already in the order used by the epilogue
+      tmem_ld128(tbase + half * 128, v);
+    }
   } else {
     if (p.epi == KL_EPI_SWIGLU) {
       // this thread's outputs o in [half*BN/4, (half+1)*BN/4): gate column
@@ -543,7 +607,7 @@ template <int BN>
 __global__ void __launch_bounds__(352, 1)
     gemm_nvfp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                          const GemmParams p) {
+                          const __grid_constant__ CUtensorMap tmap_res, const GemmParams p) {
   using C = Gemm2Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -580,6 +644,7 @@ __global__ void __launch_bounds__(352, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
+    if (p.res_prefetch) prefetch_tmap(&tmap_res);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -623,6 +688,10 @@ __global__ void __launch_bounds__(352, 1)
           tma_load_2d_pair(sb, &tmap_b, kt * 128, nb * BN + (int)rank * (BN / 2), fb);
           tma_load_2d_pair(ssfa, &tmap_sfa, 0, (mb2 * 2 + (int)rank) * p.kbn + kt * 4, fb);
           tma_load_3d_pair(ssfb, &tmap_sfb, 0, kt * 4, nb * (BN / 128), fb);
+          // the epilogue of this tile reads its residual rows: bring them
+          // into L2 now, a whole main loop ahead, instead of in the burst in
+          // which every SM's epilogue reads at once
+          if (kt == 0 && p.res_prefetch) tma_prefetch_2d(&tmap_res, nb * BN, mb2 * 256 + (int)rank * 128);
         }
         __syncwarp();
         if (++stage == C::STAGES) {
@@ -795,7 +864,16 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
                     128, 4, 0) ||
       !make_tmap_3d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.w_scales, sfb_dims, sfb_strides, sfb_box))
     return cudaErrorInvalidValue;
+  // residual rows of a tile half (BN x 128 bf16) for the L2 prefetch; when the
+  // pointer does not suit a tensor map the prefetch is skipped
+  CUtensorMap tr = ta;
+  int res_prefetch = 0;
+  if (a.epi == KL_EPI_GATED_RESIDUAL && (reinterpret_cast<uintptr_t>(a.residual) & 15) == 0 &&
+      make_tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.residual, (uint64_t)a.N, (uint64_t)a.M,
+                   (uint64_t)a.N * 2, BN, 128, 0))
+    res_prefetch = 1;
   GemmParams p;
+  p.res_prefetch = res_prefetch;
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
@@ -833,7 +911,7 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN>, ta, tb, tsa, tsb, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN>, ta, tb, tsa, tsb, tr, p);
 }
 
 template <int BN, int KS>
@@ -848,6 +926,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
                     (uint64_t)(a.K / 2), C::ROWB, BN, swz))
     return cudaErrorInvalidValue;
   GemmParams p;
+  p.res_prefetch = 0;
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
