@@ -118,6 +118,16 @@ __device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&v)[16]) {
   }
 }
 
+// floor(b / d) for a per-launch divisor d as the high word of b * r,
+// r = ceil(2^64 / d) (host: rcp64): with r = 2^64/d + e, 0 <= e < 1, the
+// product overshoots b/d by b*e/2^64 < 1/d for every b < 2^64/d, which never
+// reaches the next integer -- exact, without a 64-bit division per element.
+// d = 1 wraps r to 0, which div_rcp reads as "no division".
+__host__ __device__ __forceinline__ uint64_t rcp64(uint64_t d) { return ~0ull / d + 1; }
+__device__ __forceinline__ int64_t div_rcp(int64_t b, uint64_t r) {
+  return r ? (int64_t)__umul64hi((uint64_t)b, r) : b;
+}
+
 __device__ __forceinline__ int64_t swiglu_src_row(int64_t r, int64_t rows) {
   const int64_t g = r >> 7, i = r & 127;
   return i < 64 ? (g << 6) + i : (rows >> 1) + (g << 6) + (i - 64);
@@ -129,7 +139,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
                                                        int64_t cols, int64_t rows_padded,
                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                        float* __restrict__ gs_io, const float* __restrict__ amax,
-                                                       int mode) {
+                                                       uint64_t kbn_rcp, int mode) {
   pdl_wait();
   pdl_trigger();
   const bool mma = mode & 1, given = mode & 2, perm = mode & 4;
@@ -141,7 +151,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
   const int64_t total = rows_padded * kbn;
   if (!given && blockIdx.x == 0 && threadIdx.x == 0) *gs_io = g.gs;
   for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < total; b += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = b / kbn, kb = b - row * kbn;
+    const int64_t row = div_rcp(b, kbn_rcp), kb = b - row * kbn;
     const int64_t soff = mma ? mma_scale_offset(row, kb, cols) : row * kbn + kb;
     if (row >= rows) {  // padding rows of the MMA layout
       scales[soff] = 0;
@@ -433,7 +443,8 @@ constexpr int kFp8MaxHeads = 512;  // ncols / 128 (the launcher checks)
 // 16 elements per thread (inside one 128-wide head).
 __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t ncols,
                                                        int64_t ld, const float* __restrict__ amax,
-                                                       uint8_t* __restrict__ out, float* __restrict__ scales_out) {
+                                                       uint8_t* __restrict__ out, float* __restrict__ scales_out,
+                                                       uint64_t n16_rcp) {
   pdl_wait();
   pdl_trigger();
   const int64_t n16 = ncols >> 4;
@@ -453,7 +464,7 @@ __global__ void __launch_bounds__(256) fp8_cast_kernel(const uint16_t* __restric
   }
   __syncthreads();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / n16, c = (i - t * n16) << 4;
+    const int64_t t = div_rcp(i, n16_rcp), c = (i - t * n16) << 4;
     const float inv = inv_tab[c >> 7];
     float v[16];
     load16_bf16(x + t * ld + c, v);
@@ -516,7 +527,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols, void* cod
   const int64_t rows_padded = (mode & 1) ? ((rows + 127) / 128) * 128 : rows;
   return launch_pdl(quantize_kernel, dim3(grid_for(rows_padded * (cols / 16), 256)), dim3(256), 0, s,
                     reinterpret_cast<const uint16_t*>(x), rows, cols, rows_padded, reinterpret_cast<uint8_t*>(codes),
-                    reinterpret_cast<uint8_t*>(scales), gs_io, amax, mode);
+                    reinterpret_cast<uint8_t*>(scales), gs_io, amax, rcp64((uint64_t)(cols / 16)), mode);
 }
 
 cudaError_t launch_ln_modulate_quantize(const void* x, int64_t rows, int64_t cols, const void* shift,
@@ -604,7 +615,7 @@ cudaError_t launch_fp8_cast(const void* x, int64_t T, int64_t ncols, int64_t ld,
   if (ncols / 128 > kFp8MaxHeads) return cudaErrorInvalidValue;
   return launch_pdl(fp8_cast_kernel, dim3(grid_for(T * (ncols / 16), 256)), dim3(256), 0, s,
                     reinterpret_cast<const uint16_t*>(x), T, ncols, ld, amax, reinterpret_cast<uint8_t*>(out),
-                    scales_out);
+                    scales_out, rcp64((uint64_t)(ncols / 16)));
 }
 
 cudaError_t launch_rope_table(int64_t n_text, int64_t gh, int64_t gw, int64_t n_ref, double theta, float* cs,
