@@ -288,6 +288,42 @@ __device__ __forceinline__ void epilogue_apply(const GemmParams& p, float (&v)[B
 
 }
 
+// The gated-residual epilogue with the tile's residual rows already in
+// shared memory, brought in by TMA during the main loop as 4 boxes of 64
+// columns x 128 rows (bf16, 128-byte swizzle: the 16-byte chunk k of row r
+// sits at chunk k ^ (r & 7), so the 32 rows a warp reads at one column offset
+// hit 8 different chunk positions).  BN 256 tiles, 8 epilogue warps, half =
+// which 128 columns.
+__device__ __forceinline__ void epilogue_apply_smem(const GemmParams& p, float (&v)[128], float alpha, int64_t row,
+                                                    bool valid, int64_t n0, int half, int r, const uint8_t* es) {
+  if (!valid) return;
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] *= alpha;
+  uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + row * p.N + n0 + half * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint8_t* box = es + (2 * half + (c >> 1)) * 16384 + r * 128;
+    uint32_t rw[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 q = *reinterpret_cast<const uint4*>(box + ((((c & 1) * 4 + u) ^ (r & 7)) << 4));
+      rw[4 * u] = q.x;
+      rw[4 * u + 1] = q.y;
+      rw[4 * u + 2] = q.z;
+      rw[4 * u + 3] = q.w;
+    }
+    float gt[32];
+    load_bf16x32(p.gate + n0 + half * 128 + c * 32, gt);  // the same 64 bytes for every row: L1 hits
+    float* w = v + c * 32;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      w[2 * j] = __fmaf_rn(gt[2 * j], w[2 * j], bf16_bits_to_f32(rw[j] & 0xFFFFu));
+      w[2 * j + 1] = __fmaf_rn(gt[2 * j + 1], w[2 * j + 1], bf16_bits_to_f32(rw[j] >> 16));
+    }
+    store_bf16x32(dst + c * 32, *reinterpret_cast<float(*)[32]>(w));
+  }
+}
+
 // Drains one thread's slice of a 128 x BN accumulator (its TMEM lane group
 // at tbase) into registers: the BN/2 columns of tile half `half`, or for
 // SwiGLU the BN/4 gate and BN/4 up columns of the outputs that half owns.
@@ -575,49 +611,59 @@ __global__ void __launch_bounds__(352, 1)
 //
 // Roles (whole warps; one elected lane issues): warp 0 of both CTAs loads its
 // operand tiles and scales with cta_group::2 tensor copies that signal the
-// leader's stage barrier; on the leader, warp 10 copies each stage's scales
-// into TMEM (tcgen05.cp.cta_group::2) and warp 1 issues the MMAs, multicasting
-// its commits to both CTAs' stage-empty and accumulator-full barriers; warps
-// 2-9 of both CTAs drain their accumulator and arrive on the leader's
-// accumulator-empty barrier.
+// leader's stage barrier; warp 1 of the leader issues the scale copies into
+// TMEM (tcgen05.cp.cta_group::2) and the MMAs, multicasting its commits to
+// both CTAs' stage-empty and accumulator-full barriers; warps 2-9 of both
+// CTAs drain their accumulator and arrive on the leader's accumulator-empty
+// barrier.  Warp 10: with a staged gated epilogue (ESM) it loads each tile's
+// residual rows into shared memory one tile ahead; built with
+// KL_SF_IN_MMA=0 it copies the scales instead of warp 1.
 #ifndef KL_SF_IN_MMA
 #define KL_SF_IN_MMA 1
 #endif
 
-template <int BN>
+// ESM: the gated epilogue's residual rows are staged in shared memory (64 KB,
+// loaded by warp 10 during the main loop; one K stage fewer).
+template <int BN, bool ESM = false>
 struct Gemm2Cfg {
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = (BN / 2) * 128;
   static constexpr int SFA_BYTES = 4 * 512;
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = ESM ? 4 : (196 * 1024) / STAGE_BYTES;
+  static constexpr int EPI_BYTES = ESM ? 65536 : 0;
   static constexpr int ACC = BN == 256 ? 1 : 2;
   static constexpr uint32_t ACC_COLS = BN;
   static constexpr uint32_t SF_COLS = 16 + 16 * (BN / 128);
   static constexpr uint32_t SF_BASE = ACC * ACC_COLS;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 512;
   static_assert(SF_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "smem budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(!ESM || BN == 256, "staged epilogue: 256-column tiles");
+  static_assert(!ESM || KL_SF_IN_MMA, "the staged rows' loader is the scale-copier warp");
 };
 
-template <int BN>
+template <int BN, bool ESM>
 __global__ void __launch_bounds__(352, 1)
     gemm_nvfp4_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                           const __grid_constant__ CUtensorMap tmap_res, const GemmParams p) {
-  using C = Gemm2Cfg<BN>;
+  using C = Gemm2Cfg<BN, ESM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* epi_smem = smem + C::STAGES * C::STAGE_BYTES;  // ESM: 64 KB, 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* sf_ready = empty + C::STAGES;
   uint64_t* tfull = sf_ready + C::STAGES;  // ACC
   uint64_t* tempty = tfull + C::ACC;       // ACC (leader: 16 arrivals each)
   uint64_t* drain = tempty + C::ACC;       // 2
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* epi_full = drain + 2;          // ESM: this CTA's staged rows landed
+  uint64_t* epi_empty = epi_full + 1;      // ESM: its 8 epilogue warps are done with them
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -636,6 +682,8 @@ __global__ void __launch_bounds__(352, 1)
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(epi_full, 1);
+    mbar_init(epi_empty, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -644,7 +692,7 @@ __global__ void __launch_bounds__(352, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
-    if (p.res_prefetch) prefetch_tmap(&tmap_res);
+    if (p.res_prefetch || ESM) prefetch_tmap(&tmap_res);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -691,7 +739,7 @@ __global__ void __launch_bounds__(352, 1)
           // the epilogue of this tile reads its residual rows: bring them
           // into L2 now, a whole main loop ahead, instead of in the burst in
           // which every SM's epilogue reads at once
-          if (kt == 0 && p.res_prefetch) tma_prefetch_2d(&tmap_res, nb * BN, mb2 * 256 + (int)rank * 128);
+          if (!ESM && kt == 0 && p.res_prefetch) tma_prefetch_2d(&tmap_res, nb * BN, mb2 * 256 + (int)rank * 128);
         }
         __syncwarp();
         if (++stage == C::STAGES) {
@@ -768,8 +816,24 @@ __global__ void __launch_bounds__(352, 1)
       warp_wait(&drain[0], 0, &no_abort);
     }
   } else if (warp == 10) {
-    // ------------------------------------------------ scale copier (leader)
-    if (leader && !KL_SF_IN_MMA) {
+    if (ESM) {
+      // ------------------------------- residual rows loader (both CTAs)
+      // one tile ahead of the epilogue: once its warps are done with the
+      // previous tile's rows, this CTA's 128 residual rows of the next tile
+      int it = 0;
+      for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+        const int mb2 = tile % num_m2, nb = tile / num_m2;
+        if (!warp_wait(epi_empty, ((uint32_t)it & 1u) ^ 1u, abort_flag)) break;
+        if (elect_one()) {
+          const int y = mb2 * 256 + (int)rank * 128;
+          mbar_arrive_expect_tx(epi_full, 65536);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) tma_load_2d(epi_smem + b * 16384, &tmap_res, nb * BN + 64 * b, y, epi_full);
+        }
+        __syncwarp();
+      }
+    } else if (leader && !KL_SF_IN_MMA) {
+      // ---------------------------------------------- scale copier (leader)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -818,6 +882,7 @@ __global__ void __launch_bounds__(352, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     float v[BN / 2];
+    int it = 0;  // ESM: tiles done (phase of the staged rows)
     for (int tile = pair; tile < num_tiles; tile += npairs) {
       const int mb2 = tile % num_m2, nb = tile / num_m2;
       if (!warp_wait(&tfull[acc], acc_phase, abort_flag)) break;
@@ -832,7 +897,15 @@ __global__ void __launch_bounds__(352, 1)
         acc_phase ^= 1u;
       }
       const int64_t row = (int64_t)mb2 * 256 + rank * 128 + row_in_tile;
-      epilogue_apply<BN>(p, v, alpha, row, row < p.M, (int64_t)nb * BN, half, lane);
+      if constexpr (ESM) {
+        if (!warp_wait(epi_full, (uint32_t)it & 1u, abort_flag)) break;
+        epilogue_apply_smem(p, v, alpha, row, row < p.M, (int64_t)nb * BN, half, row_in_tile, epi_smem);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_empty);
+        ++it;
+      } else {
+        epilogue_apply<BN>(p, v, alpha, row, row < p.M, (int64_t)nb * BN, half, lane);
+      }
     }
   }
 
@@ -845,9 +918,9 @@ __global__ void __launch_bounds__(352, 1)
   }
 }
 
-template <int BN>
-static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
-  using C = Gemm2Cfg<BN>;
+template <int BN, bool ESM>
+static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s, const CUtensorMap* t_epi) {
+  using C = Gemm2Cfg<BN, ESM>;
   CUtensorMap ta, tb, tsa, tsb;
   const uint64_t kbn = (uint64_t)(a.K / 64);
   // block scales: SFA as rows of one 512-byte atom (128 x uint32), 4 atoms
@@ -864,11 +937,12 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
                     128, 4, 0) ||
       !make_tmap_3d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.w_scales, sfb_dims, sfb_strides, sfb_box))
     return cudaErrorInvalidValue;
-  // residual rows of a tile half (BN x 128 bf16) for the L2 prefetch; when the
-  // pointer does not suit a tensor map the prefetch is skipped
-  CUtensorMap tr = ta;
+  // ESM: the staged epilogue rows' map (t_epi); otherwise the residual rows
+  // of a tile half (BN x 128 bf16) for the L2 prefetch, skipped when the
+  // pointer does not suit a tensor map
+  CUtensorMap tr = ESM ? *t_epi : ta;
   int res_prefetch = 0;
-  if (a.epi == KL_EPI_GATED_RESIDUAL && (reinterpret_cast<uintptr_t>(a.residual) & 15) == 0 &&
+  if (!ESM && a.epi == KL_EPI_GATED_RESIDUAL && (reinterpret_cast<uintptr_t>(a.residual) & 15) == 0 &&
       make_tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.residual, (uint64_t)a.N, (uint64_t)a.M,
                    (uint64_t)a.N * 2, BN, 128, 0))
     res_prefetch = 1;
@@ -893,7 +967,7 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
   p.kbn = (int)kbn;
   p.num_kt = (p.kbn + 3) / 4;
   cudaError_t e =
-      cudaFuncSetAttribute(gemm_nvfp4_2sm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      cudaFuncSetAttribute(gemm_nvfp4_2sm_kernel<BN, ESM>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int pairs_max = device_sm_count() / 2;
   const int pairs = p.num_tiles < pairs_max ? p.num_tiles : pairs_max;
@@ -911,7 +985,7 @@ static cudaError_t launch_2sm(const GemmArgs& a, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN>, ta, tb, tsa, tsb, tr, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_2sm_kernel<BN, ESM>, ta, tb, tsa, tsb, tr, p);
 }
 
 template <int BN, int KS>
@@ -964,8 +1038,23 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   int bn = a.force_bn;
   if (bn == 0) bn = a.M > 128 ? ((a.N % 256 == 0) ? 512 : 384) : ((a.N % 256 == 0) ? 256 : 128);
   if ((bn == 256 || bn == 512) && a.N % 256 != 0) return cudaErrorInvalidValue;
-  if (bn == 512) return launch_2sm<256>(a, s);
-  if (bn == 384) return launch_2sm<128>(a, s);
+  if (bn == 512) {
+    // Staged epilogue rows (shared memory filled by TMA during the main loop,
+    // one K stage fewer): measured a gain only for the gated residual with a
+    // short K (the out-projection, K = 3,072: 59.4 -> 55.3 us at 8,704 rows);
+    // with K = 9,216 the lost stage costs more (60 -> 65 us), and the QKV
+    // RoPE table staged the same way was slower too (74 -> 77 us), so those
+    // keep the L2-prefetch / register epilogue.  Used when the pointer suits
+    // a tensor map.
+    CUtensorMap te;
+    bool esm = false;
+    if (a.epi == KL_EPI_GATED_RESIDUAL && a.K <= 4096 && a.residual &&
+        (reinterpret_cast<uintptr_t>(a.residual) & 15) == 0)
+      esm = make_tmap_2d(&te, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.residual, (uint64_t)a.N, (uint64_t)a.M,
+                         (uint64_t)a.N * 2, 64, 128, 128);
+    return esm ? launch_2sm<256, true>(a, s, &te) : launch_2sm<256, false>(a, s, nullptr);
+  }
+  if (bn == 384) return launch_2sm<128, false>(a, s, nullptr);
   return bn == 256 ? launch_bn<256, KL_GEMM_KSTEPS>(a, s) : launch_bn<128, KL_GEMM_KSTEPS>(a, s);
 }
 
