@@ -412,14 +412,16 @@ def measure_block(kl, wl, dev, steps, warmup, flush, world, peaks, clocks=None, 
         # end to end through the C ABI with host buffers: every step one
         # kl_joint_block_forward_host call (pinned x and modulation copied in,
         # the block, out copied back), all inside the timed events.  Steps
-        # alternate between two streams, each with its own device workspace
-        # and pinned output, so one step's host copies overlap the other's
-        # block (independent images, as a caller with a queue of them runs
-        # the API).  Each step moves several hundred MB through HBM, more
-        # than the L2 holds, so nothing carries over in L2 between steps.
+        # rotate over three streams, each with its own device workspace and
+        # pinned output: a stream runs its step's copy in, block and copy out
+        # in order, so with three in flight the copies of two steps overlap
+        # the block of the third (independent images, as a caller with a
+        # queue of them runs the API).  Each step moves several hundred MB
+        # through HBM, more than the L2 holds, so nothing carries over in L2
+        # between steps.
         x_h = inp["x"].pin_memory()
         mod_h = {n: inp[n].pin_memory() for n in MOD_NAMES}
-        nstr = 2
+        nstr = 3
         out_h = [torch.empty_like(x_h).pin_memory() for _ in range(nstr)]
         ws_h = [torch.empty(kl.lib().kl_block_host_workspace_size(T, D, H, F, kl.ATTN[wl.attn]), dtype=torch.uint8,
                             device=dev) for _ in range(nstr)]
@@ -534,8 +536,8 @@ def run_ours(args, wl):
             "e2e": {"value": round(whole_job_value(world, wl.n_tokens, args.steps, res["e2e_ms"]), 1), "unit": UNIT,
                     "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                     "via": "kl_joint_block_forward_host per step (pinned host x/modulation in, out back), steps "
-                           "alternating over two streams with a workspace each, so one step's copies overlap the "
-                           "other's block; no L2 flush (each step moves more than the L2 holds)"},
+                           "rotating over three streams with a workspace each, so the copies of two steps overlap "
+                           "the block of the third; no L2 flush (each step moves more than the L2 holds)"},
             "clocks": clk}
     sec = []
     for name in (() if args.no_secondary else SECONDARY.get(wl.name, ())):

@@ -357,8 +357,17 @@ __global__ void __launch_bounds__(256, 2) ln_stats_rows_kernel(const uint16_t* _
       amax_w = bf16x2_absmax(bf16x2_absmax(amax_w, m.z), m.w);
     }
   }
+  // one atomic per CTA (not per row): the 8 warps' maxima meet in shared memory
+  __shared__ float red[8];
   const float lmax = warp_max(bf16x2_hmax_f32(amax_w));
-  if (lane == 0 && row < rows) atomic_max_nonneg(amax, lmax);
+  if (lane == 0) red[warp] = lmax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+    atomic_max_nonneg(amax, m);
+  }
 }
 
 // Encode pass: recompute m from x (an L2 re-read) and the stored statistics,
