@@ -72,17 +72,27 @@ __global__ void __launch_bounds__(256) vc_share_kernel(const float* __restrict__
 // so they order like the values), 8 bits at a time from the top; then every
 // share above it is repaired, and of the shares equal to it the first ones
 // in index order, up to R.  mark[h][b][j] = 1 for a repaired pair.
+// SMEM: the head's n shares are held in shared memory (read from global
+// once); otherwise every pass reads them from global memory.  The bin holding
+// the R-th value is found by warp 0 (8 bins per lane, suffix sums by
+// shuffles), the index order of equal shares by a two-level shuffle scan.
+template <bool SMEM>
 __global__ void __launch_bounds__(1024) vc_topk_kernel(const float* __restrict__ w, int n, int R,
                                                        uint8_t* __restrict__ mark) {
   pdl_wait();
   pdl_trigger();
+  extern __shared__ uint32_t sv[];  // SMEM: n share bit patterns
   __shared__ unsigned int hist[256];
   __shared__ unsigned int sel[3];  // prefix bits, prefix mask, count still to place above the prefix
-  __shared__ int scan[1024];
-  const int h = blockIdx.x, tid = threadIdx.x;
+  __shared__ int wsum[32];
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* wb = reinterpret_cast<const uint32_t*>(w) + (int64_t)h * n;
   uint8_t* mk = mark + (int64_t)h * n;
-  for (int i = tid; i < n; i += blockDim.x) mk[i] = 0;
+  auto val = [&](int i) -> uint32_t { return SMEM ? sv[i] : __ldg(wb + i); };
+  for (int i = tid; i < n; i += blockDim.x) {
+    mk[i] = 0;
+    if (SMEM) sv[i] = __ldg(wb + i);
+  }
   if (R <= 0) return;
   if (R >= n) {
     __syncthreads();
@@ -94,52 +104,87 @@ __global__ void __launch_bounds__(1024) vc_topk_kernel(const float* __restrict__
     sel[1] = 0u;
     sel[2] = (unsigned)R;
   }
-  __syncthreads();
   for (int shift = 24; shift >= 0; shift -= 8) {
     if (tid < 256) hist[tid] = 0u;
     __syncthreads();
     const uint32_t pre = sel[0], pmask = sel[1];
     for (int i = tid; i < n; i += blockDim.x) {
-      const uint32_t v = __ldg(wb + i);
+      const uint32_t v = val(i);
       if ((v & pmask) == pre) atomicAdd(&hist[(v >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      unsigned int need = sel[2], acc = 0u;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (acc + hist[d] >= need) break;
-        acc += hist[d];
+    if (warp == 0) {
+      // lane l holds bins 255-8l .. 248-8l (descending); count at or above
+      // each of its bins = the sums of the lanes before it + its own prefix
+      unsigned int c[8], tot = 0u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = hist[255 - 8 * lane - q];
+        tot += c[q];
       }
-      sel[0] = pre | ((uint32_t)d << shift);
-      sel[1] = pmask | (255u << shift);
-      sel[2] = need - acc;
+      unsigned int before = tot;  // inclusive scan of the lane totals, then exclusive
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int t = __shfl_up_sync(0xffffffffu, before, off);
+        if (lane >= off) before += t;
+      }
+      before -= tot;
+      const unsigned int need = sel[2];
+      // the lane whose bins reach need: before < need <= before + tot
+      const bool mine = before < need && need <= before + tot;
+      const unsigned int who = __ballot_sync(0xffffffffu, mine);
+      if (mine && lane == __ffs(who) - 1) {
+        unsigned int acc = before;
+        int d = 255 - 8 * lane;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (acc + c[q] >= need) {
+            d = 255 - 8 * lane - q;
+            break;
+          }
+          acc += c[q];
+        }
+        sel[0] = pre | ((uint32_t)d << shift);
+        sel[1] = pmask | (255u << shift);
+        sel[2] = need - acc;
+      }
     }
     __syncthreads();
   }
   const uint32_t theta = sel[0];
   const unsigned int eq_take = sel[2];  // shares equal to theta that are repaired
-  // above theta: repaired; equal: the first eq_take in index order (a block
-  // scan over contiguous chunks of indices)
+  // above theta: repaired; equal: the first eq_take in index order (each
+  // thread a contiguous chunk of indices, counts scanned across the block)
   const int chunk = (n + blockDim.x - 1) / blockDim.x;
   const int i0 = tid * chunk, i1 = min(n, i0 + chunk);
   int eq = 0;
   for (int i = i0; i < i1; ++i) {
-    const uint32_t v = __ldg(wb + i);
+    const uint32_t v = val(i);
     if (v > theta) mk[i] = 1;
     eq += v == theta;
   }
-  scan[tid] = eq;
-  __syncthreads();
-  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-    const int t = tid >= off ? scan[tid - off] : 0;
-    __syncthreads();
-    scan[tid] += t;
-    __syncthreads();
+  int incl = eq;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
   }
-  int before = scan[tid] - eq;  // equal shares at lower indices
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int x = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, xi, off);
+      if (lane >= off) xi += t;
+    }
+    wsum[lane] = xi - x;  // equal shares in the warps before
+  }
+  __syncthreads();
+  int before = wsum[warp] + incl - eq;  // equal shares at lower indices
   for (int i = i0; i < i1; ++i) {
-    if (__ldg(wb + i) == theta) {
+    if (val(i) == theta) {
       if ((unsigned)before < eq_take) mk[i] = 1;
       ++before;
     }
@@ -257,7 +302,17 @@ cudaError_t launch_vc_select(const void* q, const void* k, int64_t ld, int64_t T
                  (const float*)v.kbar, nqb, nkt, 1.4426950408889634f / sqrtf(128.0f), v.w);
   if (e != cudaSuccess) return e;
   const int64_t R = vc_repair_count(T, budget);
-  e = launch_pdl(vc_topk_kernel, dim3((unsigned)H), dim3(1024), 0, s, (const float*)v.w, nqb * nkt, (int)R, v.mark);
+  const int n = nqb * nkt;
+  const size_t tsm = (size_t)n * sizeof(uint32_t);
+  if (tsm <= 160 * 1024) {
+    if (tsm > 48 * 1024) {
+      e = cudaFuncSetAttribute(vc_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl(vc_topk_kernel<true>, dim3((unsigned)H), dim3(1024), tsm, s, (const float*)v.w, n, (int)R, v.mark);
+  } else {
+    e = launch_pdl(vc_topk_kernel<false>, dim3((unsigned)H), dim3(1024), 0, s, (const float*)v.w, n, (int)R, v.mark);
+  }
   if (e != cudaSuccess) return e;
   return launch_pdl(vc_lists_kernel, dim3((unsigned)nqb, (unsigned)H), dim3(32), 0, s, (const uint8_t*)v.mark, nqb,
                     nqb16, nkt, list8, list16);
