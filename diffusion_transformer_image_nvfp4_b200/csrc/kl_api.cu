@@ -435,7 +435,9 @@ kl_status kl_vc_select(const void* q, const void* k, int64_t ld, int64_t T, int6
 // [ml8: float2 T*H][ml16: float2 T*H][o16: fp32 T*H*128]
 size_t kl_vc_attention_workspace_size(int64_t T, int64_t H) {
   if (T < 1 || H < 1) return 0;
-  return 2 * up256((size_t)T * H * sizeof(float2)) + up256((size_t)T * H * 128 * sizeof(float));
+  const int64_t nqb16 = (T + 127) / 128;
+  return 2 * up256((size_t)T * H * sizeof(float2)) + up256((size_t)T * H * 128 * sizeof(float)) +
+         up256((size_t)(H * nqb16 + 1) * sizeof(int));
 }
 
 static cudaError_t vc_attention(const AttnArgs& a8, const void* q, const void* k, const void* v, int64_t ld,
@@ -444,13 +446,22 @@ static cudaError_t vc_attention(const AttnArgs& a8, const void* q, const void* k
   float2* ml8 = reinterpret_cast<float2*>(ws);
   float2* ml16 = reinterpret_cast<float2*>(ws + up256((size_t)T * H * sizeof(float2)));
   float* o16 = reinterpret_cast<float*>(ws + 2 * up256((size_t)T * H * sizeof(float2)));
+  int* work = reinterpret_cast<int*>(ws + 2 * up256((size_t)T * H * sizeof(float2)) +
+                                     up256((size_t)T * H * 128 * sizeof(float)));
+  const int nqb16 = (int)((T + 127) / 128), nkt = (int)((T + 127) / 128);
+  int* work_count = work + H * nqb16;
   AttnArgs f = a8;  // the FP8 pass over the tiles that are not repaired
   f.amax = nullptr;
   f.ml_out = ml8;
   f.empty_ok = 1;
   cudaError_t e = launch_attention(f, s);
   if (e != cudaSuccess) return e;
-  AttnArgs b{};  // the BF16 pass over the repaired tiles
+  // the BF16 pass over the repaired tiles runs only the (head, 128-row
+  // block) items that have some: rows of the others keep l = 0 in ml16, which
+  // the merge reads as "no repaired part"
+  if ((e = cudaMemsetAsync(ml16, 0, (size_t)T * H * sizeof(float2), s)) != cudaSuccess) return e;
+  if ((e = launch_list_work(list16, H, nqb16, nkt, work, work_count, s)) != cudaSuccess) return e;
+  AttnArgs b{};
   b.q = q;
   b.k = k;
   b.v = v;
@@ -463,6 +474,8 @@ static cudaError_t vc_attention(const AttnArgs& a8, const void* q, const void* k
   b.ml_out = ml16;
   b.o32 = o16;
   b.empty_ok = 1;
+  b.work = work;
+  b.work_count = work_count;
   if ((e = launch_attention(b, s)) != cudaSuccess) return e;
   if ((e = launch_vc_merge(a8.out, o16, ml8, ml16, T, H, s)) != cudaSuccess) return e;
   if (!a8.amax) return cudaSuccess;

@@ -55,6 +55,8 @@ struct AttnParams {
   float2* ml_out;      // [T, H]: per row the reference maximum m and the mass l (sum 2^(t-m) of the visited keys)
   float* o32;          // [T, H*128] fp32: O written here (normalised, FP8: times s_v) instead of bf16 to out
   int empty_ok;        // a list count of 0 is allowed: the CTA only writes ml_out = (-inf, 0) for its rows
+  const int* work;     // nullable: CTA i takes item work[i] = h * gridDim.x + qblk if i < *work_count, else exits
+  const int* work_count;
 };
 
 template <bool FP8>
@@ -117,7 +119,17 @@ __global__ void __launch_bounds__(AttnCfg<FP8>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qblk = blockIdx.x, h = blockIdx.y;
+  int qblk = blockIdx.x, h = blockIdx.y;
+  if (SPARSE && p.work) {
+    // a compacted work list: the items are known only once the previous
+    // kernel is done, and a CTA past the count leaves before any setup
+    pdl_wait();
+    const int i = blockIdx.y * gridDim.x + blockIdx.x;
+    if (i >= __ldg(p.work_count)) return;
+    const int item = __ldg(p.work + i);
+    qblk = item % gridDim.x;
+    h = item / gridDim.x;
+  }
   // dense: key tiles 0..n_kv-1; sparse: the listed ones (read after pdl_wait)
   const int* kv_tiles = SPARSE ? p.kv_list + ((int64_t)h * gridDim.x + qblk) * (p.n_kv + 1) : nullptr;
   if (threadIdx.x == 0) {
@@ -512,6 +524,9 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t s) {
   p.ml_out = a.ml_out;
   p.o32 = a.o32;
   p.empty_ok = a.empty_ok;
+  p.work = a.work;
+  p.work_count = a.work_count;
+  if (a.work && !a.kv_list) return cudaErrorInvalidValue;
   const int qblocks = (int)((a.T + 128 * C::QT - 1) / (128 * C::QT));
   dim3 grid((unsigned)qblocks, (unsigned)a.H);
   auto kern = a.kv_list ? attn_kernel<FP8, true> : attn_kernel<FP8, false>;

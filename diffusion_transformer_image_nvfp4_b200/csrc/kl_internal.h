@@ -84,8 +84,13 @@ struct AttnArgs {
   float2* ml_out = nullptr;      // nullable: per (row, head) reference maximum m and mass l (partial results)
   float* o32 = nullptr;          // nullable: fp32 output instead of out (partial results)
   int empty_ok = 0;              // kv_list counts of 0 allowed (the CTA writes only ml_out)
+  const int* work = nullptr;     // nullable: only the (head, query block) items listed here, as
+  const int* work_count = nullptr;  //   h * n_qblocks + qblk, *work_count of them (CTAs past it exit)
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+// the (head, query block) items whose key-tile list is not empty, ascending
+// (h * nqb + b), and their count: one CTA, a block scan (kl_vc.cu)
+cudaError_t launch_list_work(const int* list, int64_t H, int nqb, int nkt, int* work, int* count, cudaStream_t s);
 
 // Sol-Attention key-tile selection (kl_sparse.cu)
 int sol_query_rows(bool fp8);  // rows of one attention query block: 256 (FP8) / 128 (BF16)

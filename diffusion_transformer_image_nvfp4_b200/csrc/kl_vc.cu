@@ -255,6 +255,44 @@ __global__ void __launch_bounds__(256) vc_merge_kernel(uint16_t* __restrict__ ou
   }
 }
 
+// The (head, query block) items with a non-empty key-tile list, ascending:
+// one CTA of 1024 threads, each a contiguous chunk of items, a two-level
+// shuffle scan of the counts for the output positions.
+__global__ void __launch_bounds__(1024) list_work_kernel(const int* __restrict__ list, int nitems, int stride,
+                                                         int* __restrict__ work, int* __restrict__ count) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int chunk = (nitems + blockDim.x - 1) / blockDim.x;
+  const int i0 = tid * chunk, i1 = min(nitems, i0 + chunk);
+  int c = 0;
+  for (int i = i0; i < i1; ++i) c += __ldg(list + (int64_t)i * stride) > 0;
+  int incl = c;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int x = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, xi, off);
+      if (lane >= off) xi += t;
+    }
+    wsum[lane] = xi - x;
+    if (lane == 31) *count = xi;
+  }
+  __syncthreads();
+  int pos = wsum[warp] + incl - c;
+  for (int i = i0; i < i1; ++i)
+    if (__ldg(list + (int64_t)i * stride) > 0) work[pos++] = i;
+}
+
 // ------------------------------------------------------------ host side
 struct VcWs {
   float *qbar, *kbar, *w;
@@ -316,6 +354,10 @@ cudaError_t launch_vc_select(const void* q, const void* k, int64_t ld, int64_t T
   if (e != cudaSuccess) return e;
   return launch_pdl(vc_lists_kernel, dim3((unsigned)nqb, (unsigned)H), dim3(32), 0, s, (const uint8_t*)v.mark, nqb,
                     nqb16, nkt, list8, list16);
+}
+
+cudaError_t launch_list_work(const int* list, int64_t H, int nqb, int nkt, int* work, int* count, cudaStream_t s) {
+  return launch_pdl(list_work_kernel, dim3(1), dim3(1024), 0, s, list, (int)(H * nqb), nkt + 1, work, count);
 }
 
 cudaError_t launch_vc_merge(void* out, const float* o16, const float2* ml8, const float2* ml16, int64_t T,

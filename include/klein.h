@@ -395,9 +395,10 @@ kl_status kl_joint_attention_sparse(const void* q, const void* k, const void* v,
  * ld); the two lists from kl_vc_select.  out bf16 [T, H*128]; amax_out
  * (nullable) max-accumulates max|out| (caller zero-fills).  workspace >=
  * kl_vc_attention_workspace_size(T, H) bytes, 256-byte aligned (per row and
- * head the reference maximum and mass of both parts, and the BF16 part's
- * fp32 output).  With budget 0 the result is kl_joint_attention_fp8's bit for
- * bit.
+ * head the reference maximum and mass of both parts, the BF16 part's fp32
+ * output, and the list of (head, 128-row block) items with repaired tiles:
+ * the BF16 pass runs only those).  With budget 0 the result is
+ * kl_joint_attention_fp8's bit for bit.
  */
 size_t kl_vc_workspace_size(int64_t T, int64_t H);
 kl_status kl_vc_select(const void* q, const void* k, int64_t ld, int64_t T, int64_t H, float budget, int* list_fp8,
