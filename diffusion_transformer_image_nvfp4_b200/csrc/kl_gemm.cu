@@ -27,6 +27,10 @@
 //    to registers with tcgen05.ld and released before the math, so scaling by
 //    gA*gW, the fused epilogue and the stores overlap the next tile's MMAs.
 // Smem ring: 4 (BN 256) or 6 (BN 128) stages of ~54 / 36 KB.
+// The 2-SM pair kernel further down (the one large GEMMs use) keeps these
+// roles with cta_group::2 MMAs; its scale copies are issued by the MMA warp,
+// and for a gated epilogue with K <= 4096 its warp 10 stages each tile's
+// residual rows in shared memory instead (see the comments there).
 #include "kl_common.cuh"
 #include "kl_internal.h"
 #include "../../include/klein.h"
