@@ -1,7 +1,7 @@
 """The whole joint block (kl_joint_block_forward) vs the oracle, from the raw
 inputs: rel L2 of the bf16 block output within 1e-2 with BF16 attention, and
 with FP8 attention within 3e-2 of the exact oracle and 1e-2 of the oracle's
-FP8 flash pass (the benchmark spec bars).  The residual x ~ N(0, 1) dominates the
+FP8 flash pass (the block-level bars).  The residual x ~ N(0, 1) dominates the
 output; the branches themselves are bounded stage by stage, each on the
 GPU's own previous intermediate, in test_gpu_block_stages.py.  The
 multi-reference blocks (20,992 and 21,504 tokens) compare sampled output rows
